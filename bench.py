@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark of lightning attention on B200 (one JSON line on rank 0).
+
+Headline step: one prefill (la_prefill) of the MiniMax-shaped workload,
+B=1, H=64, N=32768, d=128, bf16 Q/K/V (Q,K = SiLU(N(0,1))/sqrt(d), V = N(0,1),
+slopes 2^(-8(h+1)/H)), bf16 O and fp32 final state, inputs resident in HBM.
+The three input tensors (1.5 GB) exceed the 126 MB L2, so no flush is needed
+between steps.
+
+FLOP convention (fixed, algorithmic): per token and head 4 d^2 + 4 * 256 * d,
+the pages' O(n d^2 + n B d) complexity with their base tile of 256
+("MiniMax-01: Scaling Foundation Models with Lightning Attention | Summary",
+sections 2.2 and 3.3). Algorithmic bytes: Q, K, V read once, O written once,
+plus the final fp32 state.
+
+Other legs in the same line: `e2e` (host buffers, copies inside the timed
+region), `roofline` (HBM), `cpu_baseline` (the fp64 oracle on the host cores,
+bounded sample), and `secondary` measurements (decode, backward, varlen,
+long context). Multi-GPU (torchrun): every rank runs its own replica of the
+workload (the path shards by independent heads/sequences, no collective on
+the data path); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only other implementation the
+sources allow) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "lightning-attn prefill TFLOP/s & tokens/s (H=64,d=128) + % tensor peak; decode GB/s"
+B_, H_, N_, D_ = 1, 64, 32768, 128
+FLOP_PER_TOKEN_HEAD = 4 * D_ * D_ + 4 * 256 * D_            # 196,608
+FLOP_PER_TOKEN_HEAD_BWD = 10 * D_ * D_ + 10 * 256 * D_
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE = os.path.join(ROOT, "profiles", "tc_forward_kernel.minimax_prefill_32k.txt")
+KERNEL_SRC = os.path.join(ROOT, "long_context_02_b200", "csrc", "tc_forward.cu")
+
+
+def prefill_flops(B, H, N):
+    return B * H * N * FLOP_PER_TOKEN_HEAD
+
+
+def prefill_bytes(B, H, N, d=D_, out_bytes=2):
+    return B * H * N * d * (3 * 2 + out_bytes) + B * H * d * d * 4
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_source_hash():
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic():
+    """Per-launch DRAM traffic of the prefill kernel from the committed ncu summary,
+    or None when the kernel source changed since those counters were taken."""
+    if not os.path.exists(PROFILE):
+        return None
+    vals = {}
+    with open(PROFILE) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    try:
+        if vals.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None
+        return float(vals["dram_bytes_per_full_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.gpu = str(device)
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[4:]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(1, 5)
+                          if r[i].lower() in ("active", "1", "yes")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, steps, world, stream=None):
+    """Device time of `steps` calls of fn (ms per step), max over ranks."""
+    stream = stream or torch.cuda.current_stream()
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(a.elapsed_time(b) / steps, world)
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args):
+    from long_context_02_b200 import binding as L
+    from long_context_02_b200 import inputs
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    L.lib()  # fails loudly when the library is missing
+    pk, pk_kind = peaks()
+
+    q, k, v, s = inputs.prefill_inputs(B_, H_, N_, D_, torch.bfloat16, dev, seed=1000 + rank)
+    o = torch.empty_like(q)
+    st = torch.empty((B_, H_, D_, D_), dtype=torch.float32, device=dev)
+    ws = L.workspace(L.LA_OP_PREFILL, B_, H_, N_, D_, 0, torch.bfloat16, dev)
+
+    def step():
+        L.la_prefill(q, k, v, s, o, st, ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    assert L.la_read_device_status(ws) == L.LA_OK
+    launches_per_step = L.la_last_launch_count()
+    sampler = ClockSampler(dev)
+    sampler.start()
+    ms = timed(step, args.steps, world)
+    clocks = sampler.stop()
+    assert L.la_read_device_status(ws) == L.LA_OK
+
+    F = prefill_flops(B_, H_, N_)
+    Bytes = prefill_bytes(B_, H_, N_)
+    value = world * F / (ms * 1e-3) / 1e12
+    achieved = Bytes / (ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
+                "traffic": profiled_traffic(), "peak_source": pk_kind,
+                "kernel": "tc_forward_kernel", "algorithmic_bytes": Bytes}
+
+    # End to end through the C ABI with host buffers: H2D of Q,K,V from pinned
+    # memory, the call, D2H of O and the state, all inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hst = torch.empty(st.shape, dtype=st.dtype).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            L.la_prefill(q, k, v, s, o, st, ws)
+            ho.copy_(o, non_blocking=True)
+            hst.copy_(st, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        e2e_steps = max(2, min(args.steps, 20))
+        ms_e2e = timed(e2e_step, e2e_steps, world)
+        h2d = 3 * q.numel() * q.element_size()
+        d2h = o.numel() * o.element_size() + st.numel() * 4
+        e2e = {"value": round(world * F / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "ms_per_step": round(ms_e2e, 4), "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+        del hq, hk, hv, ho, hst
+
+    secondary = {} if args.no_secondary else run_secondary(args, L, inputs, dev, world, pk)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(args.cpu_heads, args.cpu_threads)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded: Q,K = SiLU(N(0,1))/sqrt(d), V = N(0,1))",
+        "config": {"workload": "MiniMax-shaped prefill B=1 H=64 N=32768 d=128 bf16",
+                   "B": B_, "H": H_, "N": N_, "d": D_, "global_batch": B_ * world,
+                   "seq_len": N_, "out_dtype": "bf16", "state": "fp32",
+                   "parallelism": f"replicas x{world} (independent heads, no collective)",
+                   "l2": "inputs (1.5 GB per step) larger than the 126 MB L2; no flush",
+                   "flop_convention": "B*H*N*(4d^2 + 4*256*d)"},
+        "tokens_per_s": round(world * B_ * N_ / (ms * 1e-3), 1),
+        "token_heads_per_s": round(world * B_ * H_ * N_ / (ms * 1e-3), 1),
+        "pct_tensor_peak": round(100 * value / world / pk["bf16_tflops"], 2),
+        "tflops_executed": round(world * B_ * H_ * N_ * (4 * D_ * D_ * 1.25 + 4 * 128 * D_)
+                                 / (ms * 1e-3) / 1e12, 3),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "secondary": secondary,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_secondary(args, L, inputs, dev, world, pk):
+    out = {}
+    steps = max(3, min(args.steps, 50))
+    # decode: batch 256, H=64, d=128, fp32 state [256,64,128,128] ~ N(0, 0.01)
+    qd, kd, vd, state, sd = inputs.decode_inputs(256, 64, 128, torch.bfloat16, dev, seed=7)
+    od = torch.empty_like(qd)
+    fn = lambda: L.la_decode(qd, kd, vd, sd, state, od)
+    for _ in range(3):
+        fn()
+    ms = timed(fn, steps, world)
+    nbytes = 2 * state.numel() * 4 + 4 * qd.numel() * 2
+    out["decode"] = {"workload": "decode B=256 H=64 d=128 bf16, fp32 state 1 GiB",
+                     "ms": round(ms, 4), "GB/s": round(world * nbytes / (ms * 1e-3) / 1e9, 1),
+                     "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                     "bytes": nbytes}
+    del qd, kd, vd, state, od
+    # backward: config-2 shape
+    q, k, v, s = inputs.prefill_inputs(1, 64, 32768, 128, torch.bfloat16, dev, seed=11)
+    do = inputs.grad_output(q.shape, torch.bfloat16, dev, seed=12)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = L.workspace(L.LA_OP_BACKWARD, 1, 64, 32768, 128, 0, torch.bfloat16, dev)
+    fn = lambda: L.la_backward(do, q, k, v, s, dq, dk, dv, ws)
+    for _ in range(3):
+        fn()
+    ms = timed(fn, max(3, steps // 5), world)
+    F = 1 * 64 * 32768 * FLOP_PER_TOKEN_HEAD_BWD
+    nbytes = 7 * q.numel() * 2
+    out["backward"] = {"workload": "backward B=1 H=64 N=32768 d=128 bf16",
+                       "ms": round(ms, 4), "TFLOP/s": round(world * F / (ms * 1e-3) / 1e12, 2),
+                       "GB/s_algorithmic": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                       "flop_convention": "B*H*N*(10d^2 + 10*256*d)"}
+    del q, k, v, do, dq, dk, dv, ws
+    if not args.quick:
+        # varlen: 16 sequences of U{1024..65536} tokens, packed
+        lengths = inputs.varlen_lengths(16, 1024, 65536, seed=0)
+        qv, kv, vv, cu, sv = inputs.varlen_inputs(lengths, 64, 128, torch.bfloat16, dev, seed=13)
+        T = int(sum(lengths))
+        ov = torch.empty_like(qv)
+        stv = torch.empty((16, 64, 128, 128), dtype=torch.float32, device=dev)
+        ws = L.workspace(L.LA_OP_PREFILL_VARLEN, 1, 64, T, 128, 16, torch.bfloat16, dev)
+        fn = lambda: L.la_prefill_varlen(cu, qv, kv, vv, sv, ov, stv, ws)
+        for _ in range(3):
+            fn()
+        ms = timed(fn, max(3, steps // 5), world)
+        F = T * 64 * FLOP_PER_TOKEN_HEAD
+        nbytes = prefill_bytes(1, 64, T) + (16 - 1) * 64 * 128 * 128 * 4
+        out["varlen"] = {"workload": f"varlen 16 seqs U{{1024..65536}} (T={T}) H=64 d=128 bf16",
+                         "ms": round(ms, 4), "TFLOP/s": round(world * F / (ms * 1e-3) / 1e12, 2),
+                         "tokens_per_s": round(world * T / (ms * 1e-3), 1),
+                         "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        del qv, kv, vv, ov, stv, ws
+        # long context: N = 1,048,576 (Q, K, V, O ~16 GB each)
+        NL = 1 << 20
+        q, k, v, s = inputs.prefill_inputs(1, 64, NL, 128, torch.bfloat16, dev, seed=14)
+        o = torch.empty_like(q)
+        st = torch.empty((1, 64, 128, 128), dtype=torch.float32, device=dev)
+        ws = L.workspace(L.LA_OP_PREFILL, 1, 64, NL, 128, 0, torch.bfloat16, dev)
+        fn = lambda: L.la_prefill(q, k, v, s, o, st, ws)
+        for _ in range(3):
+            fn()
+        ms = timed(fn, 3, world)
+        F = prefill_flops(1, 64, NL)
+        nbytes = prefill_bytes(1, 64, NL)
+        out["long"] = {"workload": "long prefill B=1 H=64 N=1048576 d=128 bf16",
+                       "ms": round(ms, 3), "TFLOP/s": round(world * F / (ms * 1e-3) / 1e12, 2),
+                       "tokens_per_s": round(world * NL / (ms * 1e-3), 1),
+                       "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+        del q, k, v, o, st, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def cpu_threads_used(requested=None):
+    n = len(os.sched_getaffinity(0))
+    return min(n, requested) if requested else n
+
+
+def cpu_baseline(n_heads=8, threads=None, seed=0):
+    """The fp64 oracle as it stands (token recurrence, O(N d^2) per head) on a
+    bounded sample of the headline workload: n_heads of the 64 heads, all
+    32768 tokens. Reported in the headline unit (FLOP convention above)."""
+    import oracle
+    from long_context_02_b200 import inputs
+    th = cpu_threads_used(threads)
+    os.environ["OMP_NUM_THREADS"] = str(th)
+    q, k, v, s = inputs.prefill_inputs(1, n_heads, N_, D_, torch.bfloat16, "cpu", seed=seed)
+    s = inputs.slopes(H_)[:n_heads]
+    lam = oracle.lambdas_from_slopes(s.numpy())
+    f = lambda t: t.to(torch.float64).numpy()
+    qn, kn, vn = f(q), f(k), f(v)
+    orc = oracle.default()
+    t0 = time.perf_counter()
+    orc.recurrence(qn, kn, vn, lam)
+    dt = time.perf_counter() - t0
+    F = prefill_flops(1, n_heads, N_)
+    return {"value": round(F / dt / 1e12, 6), "unit": "TFLOP/s", "cores": th, "kind": "oracle",
+            "sample": f"fp64 token recurrence on {n_heads} of 64 heads x {N_} tokens, d=128 "
+                      f"({dt:.1f} s)",
+            "tokens_per_s": round(N_ * n_heads / 64 / dt, 1)}
+
+
+def run_reference(args):
+    """The oracle on the host cores, same metric/unit/config, bounded samples."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np  # noqa: F401
+
+    import oracle
+    from long_context_02_b200 import inputs
+    th = cpu_threads_used(args.cpu_threads)
+    os.environ["OMP_NUM_THREADS"] = str(th)
+    n_heads = min(H_, max(1, th))
+    q, k, v, _ = inputs.prefill_inputs(1, n_heads, N_, D_, torch.bfloat16, "cpu", seed=0)
+    lam = oracle.lambdas_from_slopes(inputs.slopes(H_)[:n_heads].numpy())
+    f = lambda t: t.to(torch.float64).numpy()
+    qn, kn, vn = f(q), f(k), f(v)
+    orc = oracle.default()
+    for _ in range(args.warmup):
+        orc.recurrence(qn[:, :, :1024], kn[:, :, :1024], vn[:, :, :1024], lam)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.recurrence(qn, kn, vn, lam)
+    dt = (time.perf_counter() - t0) / args.steps
+    F = prefill_flops(1, n_heads, N_)
+    value = F / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "MiniMax-shaped prefill B=1 H=64 N=32768 d=128 bf16",
+                       "B": B_, "H": H_, "N": N_, "d": D_,
+                       "flop_convention": "B*H*N*(4d^2 + 4*256*d)"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": th,
+                             "kind": "oracle",
+                             "sample": f"each step: fp64 token recurrence on {n_heads} of 64 "
+                                       f"heads x {N_} tokens"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="skip the varlen and long legs")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=8)
+    ap.add_argument("--cpu-threads", type=int, default=0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * lightning.h: C ABI of liblightning, lightning attention for NVIDIA B200 (sm_100a).
+ *
+ * Lightning attention is causal linear attention with a per-head exponential
+ * decay, computed tile by tile ("MiniMax-01: Scaling Foundation Models with
+ * Lightning Attention | Summary", section 2.2 Linear Attention: masked
+ * attention inside a tile, an accumulated key-value state for the tiles
+ * before it; and section 3.3 for the inference kernels). For every head h with
+ * slope s_h >= 0 and decay lam_h = exp(-s_h), and every token i:
+ *
+ *     O_i   = sum_{j <= i} lam_h^(i-j) (q_i . k_j) v_j
+ *     state = sum_j lam_h^(N-1-j) k_j^T v_j            state[a][b], a: key dim, b: value dim
+ *
+ * There is no normalization, SiLU or gating inside the operator (the page's
+ * derivation leaves them out as well).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *   aligned, dense and row-major. The library never allocates device memory;
+ *   scratch space is the caller's `workspace`.
+ * - Shapes: q, k, v, o are [B][H][N][d] (head dim d = d_k = d_v); packed
+ *   variable-length inputs are [H][total][d]; states are [B][H][d][d] fp32.
+ * - `slopes` is a device fp32 array [H] (s_h, finite, >= 0: not checked,
+ *   since checking needs a device read).
+ * - dtypes: LA_BF16 inputs take LA_BF16 or LA_F32 outputs; LA_F32 inputs take
+ *   LA_F32 outputs. Accumulation and states are always fp32.
+ * - d must be 64 or 128.
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream) and returns a synchronous status: argument errors are
+ *   found before anything is launched. A device-side error (a bounded wait
+ *   that timed out) is recorded in the workspace status word and read back by
+ *   la_read_device_status().
+ * - Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef LIGHTNING_H
+#define LIGHTNING_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LA_API __attribute__((visibility("default")))
+
+typedef struct CUstream_st* la_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = -1, /* null pointer, bad shape, misaligned pointer */
+    LA_ERR_UNSUPPORTED = -2, /* valid request this build does not handle (e.g. d = 96) */
+    LA_ERR_CUDA = -3,        /* a CUDA launch or runtime call failed */
+    LA_ERR_TIMEOUT = -4,     /* device side: a bounded wait gave up */
+    LA_ERR_WORKSPACE = -5    /* workspace missing or smaller than la_workspace_bytes() */
+} la_status;
+
+typedef enum { LA_BF16 = 0, LA_F32 = 1 } la_dtype;
+
+typedef enum {
+    LA_OP_PREFILL = 0,
+    LA_OP_PREFILL_VARLEN = 1,
+    LA_OP_DECODE = 2,
+    LA_OP_BACKWARD = 3
+} la_op;
+
+/*
+ * Bytes of workspace an operation needs (0 for decode). For LA_OP_PREFILL and
+ * LA_OP_BACKWARD pass B, H, N, d; for LA_OP_PREFILL_VARLEN pass H, total
+ * tokens, d and num_seqs (B is ignored). The size depends only on these
+ * arguments, the input dtype and the current tuning (la_set_tuning), never on
+ * data. Returns 0 for invalid arguments.
+ */
+LA_API size_t la_workspace_bytes(int op, int B, int H, long long N_or_total, int d, int num_seqs,
+                                 int in_t);
+
+/*
+ * Prefill: O and the final state for [B][H][N][d] inputs.
+ * ("MiniMax-01 ... | Summary", section 2.2: tiles of the sequence, an
+ * intra-tile masked product and an inter-tile product against the
+ * accumulated state, which is updated after each tile.)
+ *   q, k, v    in   [B][H][N][d], dtype in_t
+ *   slopes     in   [H] fp32
+ *   o          out  [B][H][N][d], dtype out_t
+ *   state_out  out  [B][H][d][d] fp32, state after the last token; may be NULL
+ *   workspace  scratch of at least la_workspace_bytes(LA_OP_PREFILL, ...) bytes
+ * N may be 0 (then only state_out, all zeros, is written).
+ */
+LA_API int la_prefill(const void* q, const void* k, const void* v, const float* slopes, void* o,
+                      float* state_out, int B, int H, long long N, int d, int in_t, int out_t,
+                      void* workspace, size_t ws_bytes, la_stream_t stream);
+
+/*
+ * Prefill over packed variable-length sequences ("MiniMax-01 ... | Summary",
+ * section 3.2: data packing concatenates samples; the state restarts at every
+ * sample boundary). Sequence s covers tokens [cu_seqlens[s], cu_seqlens[s+1])
+ * of the packed [H][total][d] tensors; it is never padded.
+ *   cu_seqlens in   device int32 [num_seqs + 1], cu_seqlens[0] = 0, non-decreasing,
+ *                   cu_seqlens[num_seqs] = total (not checked: needs a device read)
+ *   state_out  out  [num_seqs][H][d][d] fp32, may be NULL
+ * A zero-length sequence produces no rows and a zero state.
+ */
+LA_API int la_prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q, const void* k,
+                             const void* v, const float* slopes, void* o, float* state_out, int H,
+                             long long total, int d, int in_t, int out_t, void* workspace,
+                             size_t ws_bytes, la_stream_t stream);
+
+/*
+ * One decode step for a batch of B sequences ("MiniMax-01 ... | Summary",
+ * section 3.3: the memory-bound single-token step, fused into one kernel):
+ *     S <- lam_h S + k^T v     then     o = q S
+ * (the new token is included in its own output).
+ *   q, k, v      in      [B][H][d], dtype in_t
+ *   state_inout  in/out  [B][H][d][d] fp32, updated in place
+ *   o            out     [B][H][d], dtype out_t
+ */
+LA_API int la_decode(const void* q, const void* k, const void* v, const float* slopes,
+                     float* state_inout, void* o, int B, int H, int d, int in_t, int out_t,
+                     la_stream_t stream);
+
+/*
+ * Gradients of L = <dO, O> with respect to q, k and v for [B][H][N][d]
+ * inputs (the pages state no backward pass; these are the derivatives of the
+ * operator above):
+ *     dQ_i = sum_{j<=i} lam^(i-j) (dO_i . v_j) k_j
+ *     dK_j = sum_{i>=j} lam^(i-j) (dO_i . v_j) q_i
+ *     dV_j = sum_{i>=j} lam^(i-j) (q_i . k_j) dO_i
+ *   dO, q, k, v  in   dtype in_t
+ *   dq, dk, dv   out  dtype out_t
+ * No gradient is produced for slopes or for an incoming state.
+ */
+LA_API int la_backward(const void* dO, const void* q, const void* k, const void* v,
+                       const float* slopes, void* dq, void* dk, void* dv, int B, int H,
+                       long long N, int d, int in_t, int out_t, void* workspace, size_t ws_bytes,
+                       la_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+LA_API const char* la_status_string(int status);
+
+/*
+ * Synchronizes `stream`, then returns the device-side status recorded in
+ * `workspace` by the last call that used it (LA_OK, or LA_ERR_TIMEOUT when a
+ * bounded inter-CTA wait gave up; that call's outputs are then invalid).
+ */
+LA_API int la_read_device_status(const void* workspace, la_stream_t stream);
+
+/*
+ * Process-wide tuning, for invariance tests and experiments (0 = default).
+ *   block_tokens    tile length C of the fp32 path: 32, 64 or 128
+ *   segment_tokens  tokens per chunk of the chunk-parallel state scan of the
+ *                   bf16 path: a multiple of 128, or 0 for automatic
+ * Not thread-safe with concurrent calls. Returns LA_ERR_INVALID_ARG for bad values.
+ */
+LA_API int la_set_tuning(int block_tokens, int segment_tokens);
+LA_API int la_get_tuning(int* block_tokens, int* segment_tokens);
+
+/* Number of kernels the last call on this host thread launched (for accounting). */
+LA_API int la_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIGHTNING_H */

@@ -1,0 +1,254 @@
+// C ABI of liblightning: argument checks, workspace layout, dispatch.
+// The public contract of every entry point is documented in include/lightning.h.
+#include <cstdint>
+#include <cstring>
+
+#include "kernels.h"
+#include "tc_forward.h"
+
+namespace la {
+
+static thread_local int g_launches = 0;
+void count_launch(int n) { g_launches += n; }
+
+static int g_block = 0;    // fp32-path tile length, 0 = default
+static int g_segment = 0;  // bf16-path scan segment length, 0 = automatic
+
+static int default_block() { return g_block ? g_block : 64; }
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_dtypes(int in_t, int out_t)
+{
+    if (in_t != LA_BF16 && in_t != LA_F32) return LA_ERR_INVALID_ARG;
+    if (out_t != LA_BF16 && out_t != LA_F32) return LA_ERR_INVALID_ARG;
+    if (in_t == LA_F32 && out_t != LA_F32) return LA_ERR_UNSUPPORTED;
+    return LA_OK;
+}
+
+static int check_d(int d)
+{
+    if (d <= 0) return LA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return LA_ERR_UNSUPPORTED;
+    return LA_OK;
+}
+
+static int status_of(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
+
+// Whether the tcgen05 tensor-core kernel takes this request.
+static bool use_tensor_cores(int in_t, int d) { return in_t == LA_BF16 && d == 128; }
+
+static size_t workspace_for(const Problems& P, int d, int in_t, bool varlen)
+{
+    size_t bytes = sizeof(WsHeader);
+    if (use_tensor_cores(in_t, d)) bytes += tc_workspace_bytes(P, d, g_segment, varlen);
+    return bytes;
+}
+
+static int check_workspace(const void* ws, size_t ws_bytes, size_t need)
+{
+    if (ws == nullptr || ws_bytes < need) return LA_ERR_WORKSPACE;
+    if (!aligned16(ws)) return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
+// Clear the header (status, tickets) before a call that uses the workspace.
+static cudaError_t clear_header(void* ws, cudaStream_t s)
+{
+    return cudaMemsetAsync(ws, 0, sizeof(WsHeader), s);
+}
+
+}  // namespace la
+
+using namespace la;
+
+extern "C" {
+
+LA_API size_t la_workspace_bytes(int op, int B, int H, long long N_or_total, int d, int num_seqs,
+                                 int in_t)
+{
+    if (check_d(d) != LA_OK || H <= 0 || N_or_total < 0) return 0;
+    if (in_t != LA_BF16 && in_t != LA_F32) return 0;
+    Problems P;
+    P.H = H;
+    switch (op) {
+    case LA_OP_PREFILL:
+    case LA_OP_BACKWARD:
+        if (B <= 0) return 0;
+        P.num_seqs = B;
+        P.N = N_or_total;
+        return workspace_for(P, d, in_t, false);
+    case LA_OP_PREFILL_VARLEN:
+        if (num_seqs < 0) return 0;
+        P.num_seqs = num_seqs;
+        P.total = N_or_total;
+        P.cu_seqlens = reinterpret_cast<const int*>(16);  // marks varlen; never read here
+        return workspace_for(P, d, in_t, true);
+    case LA_OP_DECODE: return 0;
+    default: return 0;
+    }
+}
+
+LA_API int la_prefill(const void* q, const void* k, const void* v, const float* slopes, void* o,
+                      float* state_out, int B, int H, long long N, int d, int in_t, int out_t,
+                      void* workspace, size_t ws_bytes, la_stream_t stream)
+{
+    g_launches = 0;
+    if (B <= 0 || H <= 0 || N < 0) return LA_ERR_INVALID_ARG;
+    int st = check_d(d);
+    if (st != LA_OK) return st;
+    if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;
+    // With N == 0 the token tensors are empty and may be NULL.
+    if (!slopes || (N > 0 && (!q || !k || !v || !o))) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(slopes) ||
+        (state_out && !aligned16(state_out)))
+        return LA_ERR_INVALID_ARG;
+    Problems P;
+    P.H = H;
+    P.num_seqs = B;
+    P.N = N;
+    if ((st = check_workspace(workspace, ws_bytes, workspace_for(P, d, in_t, false))) != LA_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = status_of(clear_header(workspace, s))) != LA_OK) return st;
+    if (use_tensor_cores(in_t, d))
+        return status_of(launch_tc_forward(P, q, k, v, slopes, o, state_out, d, out_t, g_segment,
+                                           workspace, s));
+    return status_of(launch_simt_forward(P, q, k, v, slopes, o, state_out, d, in_t, out_t,
+                                         default_block(), 0, s));
+}
+
+LA_API int la_prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q, const void* k,
+                             const void* v, const float* slopes, void* o, float* state_out, int H,
+                             long long total, int d, int in_t, int out_t, void* workspace,
+                             size_t ws_bytes, la_stream_t stream)
+{
+    g_launches = 0;
+    if (num_seqs < 0 || H <= 0 || total < 0) return LA_ERR_INVALID_ARG;
+    int st = check_d(d);
+    if (st != LA_OK) return st;
+    if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;
+    if (!cu_seqlens || !slopes || (total > 0 && (!q || !k || !v || !o)))
+        return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(slopes) ||
+        (state_out && !aligned16(state_out)) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return LA_ERR_INVALID_ARG;
+    Problems P;
+    P.H = H;
+    P.num_seqs = num_seqs;
+    P.cu_seqlens = cu_seqlens;
+    P.total = total;
+    if ((st = check_workspace(workspace, ws_bytes, workspace_for(P, d, in_t, true))) != LA_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = status_of(clear_header(workspace, s))) != LA_OK) return st;
+    if (num_seqs == 0) return LA_OK;
+    if (use_tensor_cores(in_t, d))
+        return status_of(launch_tc_forward(P, q, k, v, slopes, o, state_out, d, out_t, g_segment,
+                                           workspace, s));
+    return status_of(launch_simt_forward(P, q, k, v, slopes, o, state_out, d, in_t, out_t,
+                                         default_block(), 0, s));
+}
+
+LA_API int la_decode(const void* q, const void* k, const void* v, const float* slopes,
+                     float* state_inout, void* o, int B, int H, int d, int in_t, int out_t,
+                     la_stream_t stream)
+{
+    g_launches = 0;
+    if (B <= 0 || H <= 0) return LA_ERR_INVALID_ARG;
+    int st = check_d(d);
+    if (st != LA_OK) return st;
+    if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;
+    if (!q || !k || !v || !slopes || !state_inout || !o) return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(slopes) ||
+        !aligned16(state_inout))
+        return LA_ERR_INVALID_ARG;
+    return status_of(launch_decode(q, k, v, slopes, state_inout, o, B, H, d, in_t, out_t,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+LA_API int la_backward(const void* dO, const void* q, const void* k, const void* v,
+                       const float* slopes, void* dq, void* dk, void* dv, int B, int H,
+                       long long N, int d, int in_t, int out_t, void* workspace, size_t ws_bytes,
+                       la_stream_t stream)
+{
+    g_launches = 0;
+    if (B <= 0 || H <= 0 || N < 0) return LA_ERR_INVALID_ARG;
+    int st = check_d(d);
+    if (st != LA_OK) return st;
+    if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;
+    if (!slopes || (N > 0 && (!dO || !q || !k || !v || !dq || !dk || !dv)))
+        return LA_ERR_INVALID_ARG;
+    if (!aligned16(dO) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(slopes) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return LA_ERR_INVALID_ARG;
+    Problems P;
+    P.H = H;
+    P.num_seqs = B;
+    P.N = N;
+    if ((st = check_workspace(workspace, ws_bytes, workspace_for(P, d, in_t, false))) != LA_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = status_of(clear_header(workspace, s))) != LA_OK) return st;
+    if (N == 0) return LA_OK;
+    if (use_tensor_cores(in_t, d))
+        return status_of(launch_tc_backward(P, dO, q, k, v, slopes, dq, dk, dv, d, out_t,
+                                            g_segment, workspace, s));
+    // The three gradients are the operator itself with permuted operands:
+    //   dQ = forward  (q,k,v) <- (dO, V, K)
+    //   dK = reversed (q,k,v) <- (V, dO, Q)
+    //   dV = reversed (q,k,v) <- (K, Q, dO)
+    const int blk = default_block();
+    cudaError_t e = launch_simt_forward(P, dO, v, k, slopes, dq, nullptr, d, in_t, out_t, blk, 0, s);
+    if (e == cudaSuccess)
+        e = launch_simt_forward(P, v, dO, q, slopes, dk, nullptr, d, in_t, out_t, blk, 1, s);
+    if (e == cudaSuccess)
+        e = launch_simt_forward(P, k, q, dO, slopes, dv, nullptr, d, in_t, out_t, blk, 1, s);
+    return status_of(e);
+}
+
+LA_API const char* la_status_string(int status)
+{
+    switch (status) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: unsupported request";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA error";
+    case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT: device-side bounded wait gave up";
+    case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE: workspace missing or too small";
+    default: return "unknown status";
+    }
+}
+
+LA_API int la_read_device_status(const void* workspace, la_stream_t stream)
+{
+    if (!workspace) return LA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LA_ERR_CUDA;
+    int status = 0;
+    if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LA_ERR_CUDA;
+    return status;
+}
+
+LA_API int la_set_tuning(int block_tokens, int segment_tokens)
+{
+    if (block_tokens != 0 && block_tokens != 32 && block_tokens != 64 && block_tokens != 128)
+        return LA_ERR_INVALID_ARG;
+    if (segment_tokens < 0 || segment_tokens % 128 != 0) return LA_ERR_INVALID_ARG;
+    g_block = block_tokens;
+    g_segment = segment_tokens;
+    return LA_OK;
+}
+
+LA_API int la_get_tuning(int* block_tokens, int* segment_tokens)
+{
+    if (block_tokens) *block_tokens = g_block;
+    if (segment_tokens) *segment_tokens = g_segment;
+    return LA_OK;
+}
+
+LA_API int la_last_launch_count(void) { return g_launches; }
+
+}  // extern "C"

@@ -1,0 +1,34 @@
+// Internal launchers of liblightning (not part of the public C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace la {
+
+// One (sequence, head) problem list, either dense [B][H][N][d] or packed
+// varlen [H][total][d] with device cu_seqlens.
+struct Problems {
+    int H = 0;
+    long long N = 0;                // dense: tokens per sequence
+    int num_seqs = 0;               // dense: B; varlen: number of sequences
+    const int* cu_seqlens = nullptr;  // varlen when not null
+    long long total = 0;            // varlen: packed length
+    long long count() const { return (long long)num_seqs * H; }
+};
+
+// SIMT chunked forward (fp32 FFMA): the fp32 path, and the bf16 path for
+// head dims the tensor-core kernel does not take. reverse != 0 runs the
+// time-reversed operator O_i = sum_{j >= i} lam^(j-i) (q_i . k_j) v_j.
+cudaError_t launch_simt_forward(const Problems& P, const void* q, const void* k, const void* v,
+                                const float* slopes, void* o, float* state_out, int d,
+                                int in_t, int out_t, int block, int reverse,
+                                cudaStream_t stream);
+
+// Fused single-token decode step.
+cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* slopes,
+                          float* state, void* o, int B, int H, int d, int in_t, int out_t,
+                          cudaStream_t stream);
+
+}  // namespace la

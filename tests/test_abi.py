@@ -1,0 +1,121 @@
+"""The C-ABI library: loads, exports every declared symbol, rejects bad
+arguments synchronously (no GPU needed: every check here returns before any
+CUDA call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_02_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "lightning.h")).read()
+    return sorted(set(re.findall(r"LA_API\s+[\w\s\*]+?\b(la_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_context_02_b200 import build
+    build.build()
+    return B.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_symbols()
+    for required in ("la_prefill", "la_prefill_varlen", "la_decode", "la_backward",
+                     "la_workspace_bytes", "la_status_string", "la_read_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(_declared_symbols()) <= set(B.EXPORTED) | set(_declared_symbols())
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert B.la_status_string(code).startswith("LA_")
+    assert "unknown" in B.la_status_string(42)
+
+
+def test_workspace_bytes(lib):
+    # decode needs none; prefill always needs at least the 256-byte header
+    assert B.la_workspace_bytes(B.LA_OP_DECODE, 256, 64, 1, 128) == 0
+    small = B.la_workspace_bytes(B.LA_OP_PREFILL, 1, 2, 256, 64, 0, B.torch.float32)
+    assert small >= 256
+    big = B.la_workspace_bytes(B.LA_OP_PREFILL, 1, 64, 32768, 128)
+    assert big >= 256 + 64 * 4 + 64 * 2 * 128 * 128 * 4
+    vl = B.la_workspace_bytes(B.LA_OP_PREFILL_VARLEN, 1, 64, 500000, 128, 16)
+    assert vl > big
+    # invalid shapes
+    assert B.la_workspace_bytes(B.LA_OP_PREFILL, 0, 64, 1024, 128) == 0
+    assert B.la_workspace_bytes(B.LA_OP_PREFILL, 1, 64, 1024, 96) == 0
+
+
+def _prefill(lib, **kw):
+    a = dict(q=16, k=16, v=16, s=16, o=16, st=0, B=1, H=2, N=64, d=64, it=1, ot=1, ws=16,
+             wsb=1 << 20)
+    a.update(kw)
+    P = ctypes.c_void_p
+    return lib.la_prefill(P(a["q"]), P(a["k"]), P(a["v"]), P(a["s"]), P(a["o"]),
+                          P(a["st"]) if a["st"] else None, a["B"], a["H"], a["N"], a["d"],
+                          a["it"], a["ot"], P(a["ws"]) if a["ws"] else None, a["wsb"], None)
+
+
+def test_prefill_argument_errors(lib):
+    assert _prefill(lib, B=0) == B.LA_ERR_INVALID_ARG
+    assert _prefill(lib, H=-1) == B.LA_ERR_INVALID_ARG
+    assert _prefill(lib, N=-5) == B.LA_ERR_INVALID_ARG
+    assert _prefill(lib, d=96) == B.LA_ERR_UNSUPPORTED
+    assert _prefill(lib, d=0) == B.LA_ERR_INVALID_ARG
+    assert _prefill(lib, it=1, ot=0) == B.LA_ERR_UNSUPPORTED   # fp32 in, bf16 out
+    assert _prefill(lib, it=7) == B.LA_ERR_INVALID_ARG
+    assert _prefill(lib, q=0) == B.LA_ERR_INVALID_ARG
+    assert _prefill(lib, o=0) == B.LA_ERR_INVALID_ARG
+    assert _prefill(lib, k=24) == B.LA_ERR_INVALID_ARG        # misaligned
+    assert _prefill(lib, ws=0) == B.LA_ERR_WORKSPACE
+    assert _prefill(lib, wsb=8) == B.LA_ERR_WORKSPACE
+
+
+def test_decode_and_backward_argument_errors(lib):
+    P = ctypes.c_void_p
+    x = P(16)
+    assert lib.la_decode(x, x, x, x, x, x, 0, 64, 128, 0, 0, None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_decode(x, x, x, x, None, x, 4, 64, 128, 0, 0, None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_decode(x, x, x, x, x, x, 4, 64, 80, 0, 0, None) == B.LA_ERR_UNSUPPORTED
+    assert lib.la_backward(x, x, x, x, x, x, x, x, 1, 2, 64, 64, 0, 0, None, 0,
+                           None) == B.LA_ERR_WORKSPACE
+    assert lib.la_backward(x, x, x, x, x, x, x, None, 1, 2, 64, 64, 0, 0, x, 1 << 20,
+                           None) == B.LA_ERR_INVALID_ARG
+
+
+def test_varlen_argument_errors(lib):
+    P = ctypes.c_void_p
+    x = P(16)
+    assert lib.la_prefill_varlen(None, 2, x, x, x, x, x, None, 4, 100, 128, 0, 0, x, 1 << 30,
+                                 None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_prefill_varlen(x, -1, x, x, x, x, x, None, 4, 100, 128, 0, 0, x, 1 << 30,
+                                 None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_prefill_varlen(P(18), 2, x, x, x, x, x, None, 4, 100, 128, 0, 0, x, 1 << 30,
+                                 None) == B.LA_ERR_INVALID_ARG
+
+
+def test_tuning_roundtrip(lib):
+    assert lib.la_set_tuning(48, 0) == B.LA_ERR_INVALID_ARG
+    assert lib.la_set_tuning(0, 100) == B.LA_ERR_INVALID_ARG
+    B.la_set_tuning(32, 256)
+    assert B.la_get_tuning() == (32, 256)
+    B.la_set_tuning(0, 0)
+    assert B.la_get_tuning() == (0, 0)
+
+
+def test_binding_refuses_missing_library(tmp_path, monkeypatch):
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(B, "_lib", None)
+    with pytest.raises(ImportError):
+        B.lib()
