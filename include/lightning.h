@@ -157,6 +157,39 @@ LA_API int la_get_tuning(int* block_tokens, int* segment_tokens);
 /* Number of kernels the last call on this host thread launched (for accounting). */
 LA_API int la_last_launch_count(void);
 
+/*
+ * Size in bytes of the scratch array built into the library for
+ * la_prefill_noalloc (16 MiB).
+ */
+#define LA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/*
+ * la_prefill without a caller-supplied workspace. The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory (a C or embedded host program without a device allocator, a
+ * plugin whose host application forbids allocations after start-up, a
+ * latency-critical loop that must not call cudaMalloc).
+ *
+ * Same arguments, results and errors as la_prefill, minus the workspace. The
+ * scratch is a fixed array of LA_NOALLOC_SCRATCH_BYTES in device memory that
+ * every GPU which loads the library holds until the process exits. Requests
+ * whose la_workspace_bytes(LA_OP_PREFILL, ...) exceeds that size are refused
+ * with LA_ERR_WORKSPACE before any GPU work (for bf16 inputs with d = 128 the
+ * scratch covers up to 127 (sequence, head) pairs, B*H; the fp32 path needs
+ * only a few hundred bytes).
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture. The
+ * function allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine). All calls share the one array, which keeps the last call's
+ * contents; each call clears what must start at zero on its own stream. Calls
+ * that overlap on the GPU (other streams, other host threads) race on the
+ * array: serialize them.
+ */
+LA_API int la_prefill_noalloc(const void* q, const void* k, const void* v, const float* slopes,
+                              void* o, float* state_out, int B, int H, long long N, int d,
+                              int in_t, int out_t, la_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,7 +25,7 @@ LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE, LA_OP_BACKWARD = 0, 1, 2, 3
 
 EXPORTED = ["la_workspace_bytes", "la_prefill", "la_prefill_varlen", "la_decode", "la_backward",
             "la_status_string", "la_read_device_status", "la_set_tuning", "la_get_tuning",
-            "la_last_launch_count"]
+            "la_last_launch_count", "la_prefill_noalloc"]
 
 _lib = None
 
@@ -57,9 +57,10 @@ def lib():
         L.la_set_tuning.argtypes = [I, I]
         L.la_get_tuning.argtypes = [ctypes.POINTER(I), ctypes.POINTER(I)]
         L.la_last_launch_count.argtypes = []
+        L.la_prefill_noalloc.argtypes = [P, P, P, P, P, P, I, I, LL, I, I, I, P]
         for f in ("la_prefill", "la_prefill_varlen", "la_decode", "la_backward",
                   "la_read_device_status", "la_set_tuning", "la_get_tuning",
-                  "la_last_launch_count"):
+                  "la_last_launch_count", "la_prefill_noalloc"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -129,6 +130,15 @@ def la_backward(dout, q, k, v, slopes, dq, dk, dv, ws, stream=None):
     _check("la_backward", lib().la_backward(
         _ptr(dout), _ptr(q), _ptr(k), _ptr(v), _ptr(slopes), _ptr(dq), _ptr(dk), _ptr(dv),
         B, H, N, d, _dt(q), _dt(dq), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def la_prefill_noalloc(q, k, v, slopes, o, state_out, stream=None):
+    """la_prefill on the library's built-in scratch (for callers that cannot
+    allocate device memory; see include/lightning.h)."""
+    B, H, N, d = q.shape
+    _check("la_prefill_noalloc", lib().la_prefill_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(slopes), _ptr(o), _ptr(state_out), B, H, N, d,
+        _dt(q), _dt(o), _stream(stream)))
 
 
 def la_read_device_status(ws, stream=None) -> int:
