@@ -23,7 +23,7 @@
 //     counter) and publish S_incl = lam^len S_prev + S_loc: the scan combine
 //     (a1, S1) o (a2, S2) = (a1 a2, a2 S1 + S2).
 //   phase C: run the segment's 128-token blocks from S_in = S_prev:
-//     MMA1  SB  = Q K^T                     (bf16 inputs, fp32 in TMEM)
+//     MMA1  SB  = Q K^T                     (fp32 in TMEM)
 //     E_P   P   = SB * lam^(i-j) [j<=i]      (fp16, written back into TMEM)
 //     MMA2  OI  = P V                       (A operand from TMEM)
 //     MMA3  OE  = Q S                       (S: fp32 state kept in registers)
@@ -34,20 +34,22 @@
 // Only non-negative decay exponents <= the block length appear, so nothing
 // overflows; terms that underflow are below fp32 resolution of the result.
 //
-// Precision. The operands the kernel creates itself (P, the state copy, the
-// decayed keys) and the ones it reuses in those products (Q, V) are fp16 with
-// exact power-of-two scaling, so their relative rounding is 2^-11 (bf16 would
-// be 2^-8, too coarse for a max error of 1e-2 of rms) while fp16's narrow
-// exponent range never bites: every V row, P row and Q row is scaled so its
-// largest magnitude is in [1, 2); V's row scales are folded into P's columns
-// and into the decayed keys; the decayed-key tile has one scale; each column
-// of the state copy has its own scale (the state is held transposed, one
-// value column per thread, so that is a thread-local choice). All scales are
-// undone in fp32 in the epilogues.
+// Precision. Every tensor-core operand is fp16 with exact power-of-two
+// scaling: the relative rounding of the operands the kernel forms itself (P,
+// the state copy, the decayed keys) is 2^-11 (bf16 would be 2^-8, too coarse
+// for a max error of 1e-2 of rms), and fp16's narrow exponent range never
+// bites. As tiles land, converter warps rewrite Q (one scale per row), K and
+// V (one scale per tile) as fp16 in [1, 2) magnitude; the bf16 -> fp16 step
+// is exact. Then Q K^T is bounded by 512, so P needs no rescaling, and the
+// decayed keys are bounded by the K tile. Each column of the state copy has
+// its own scale (the state is held transposed, one value column per thread,
+// so that is a thread-local choice). All scales are undone in fp32 in the
+// epilogues.
 //
-// Warp roles (12 warps): 0 TMA producer, 1 MMA issuer (also owns TMEM),
-// 2-3 idle, 4-7 "PK" epilogue (V/Q conversion, E_P, E_K), 8-11 "OS" epilogue
-// (E_O, E_S, scan). TMEM: 512 columns = SB/P | OI | OE | DS^T, 128 lanes.
+// Warp roles (16 warps, 4 warpgroups): warp 0 TMA producer, warp 1 MMA
+// issuer (also owns TMEM), warps 2-3 idle; 4-7 converters (fp16 Q, K, V as
+// tiles land); 8-11 "PE" (E_P and E_K after Q K^T); 12-15 "OS" (E_O, E_S and
+// the scan). TMEM: 512 columns = SB/P | OI | OE | DS^T, 128 lanes.
 // Shared memory: 2 stages x (Q, K, V) 128x128 16-bit tiles + the fp16 state
 // copy, all in the 128-byte-swizzled layout TMA writes.
 //
@@ -68,13 +70,13 @@ namespace tc {
 
 constexpr int D = 128;                           // head dim (d_k = d_v)
 constexpr int C = 128;                           // tokens per block
-constexpr int NUM_THREADS = 384;                 // 3 warpgroups
+constexpr int NUM_THREADS = 512;                 // 4 warpgroups
 // Register split (setmaxnreg, which ptxas also uses to allocate each role):
-// launched at 65536 / 384 -> 168 per thread, i.e. 64512 per CTA. The control
-// warpgroup drops to 64, the PK group keeps 168, the OS group rises to 232:
-// 128 * (64 + 168 + 232) = 59392 <= 64512, and per SM sub-partition (one warp
-// of each group) 32 * (64 + 168 + 232) = 14848 <= 16384.
-constexpr int REGS_CTRL = 64, REGS_OS = 232;
+// launched at 65536 / 512 = 128 per thread, i.e. 65536 per CTA. The control
+// warpgroup drops to 64, the converters to 104, the PE group to 112, the OS
+// group rises to 232: 128 * (64 + 104 + 112 + 232) = 65536, and per SM
+// sub-partition (one warp of each group) 32 * 512 = 16384.
+constexpr int REGS_CTRL = 64, REGS_CV = 104, REGS_PE = 112, REGS_OS = 232;
 constexpr uint32_t BOX_BYTES = 128 * 64 * 2;     // one TMA box: 128 rows x 64 bf16
 constexpr uint32_t TILE_BYTES = 2 * BOX_BYTES;   // 128 x 128 bf16
 constexpr uint32_t STAGE_BYTES = 3 * TILE_BYTES; // Q, K, V
@@ -86,10 +88,11 @@ constexpr unsigned long long FLAG_LIMIT_NS = 2000000000ull;
 constexpr unsigned long long DRAIN_LIMIT_NS = 200000000ull;
 
 enum {
-    B_FULL0, B_FULL1, B_EMPTY0, B_EMPTY1, B_KT0, B_KT1, B_SBLK_FULL, B_SB_FREE, B_P_READY,
-    B_O_FULL, B_O_EMPTY, B_DS_FULL, B_DS_EMPTY, B_S_READY, B_ITEM_FULL0, B_ITEM_FULL1,
-    B_ITEM_EMPTY0, B_ITEM_EMPTY1, B_FIN, B_PK_SYNC, B_OS_SYNC, B_Q_READY, B_KM_FULL0,
-    B_KM_FULL1, B_KM_EMPTY0, B_KM_EMPTY1, NUM_BARS
+    B_FULL0, B_FULL1, B_EMPTY0, B_EMPTY1, B_CONV0, B_CONV1, B_KT0, B_KT1, B_SBLK_FULL,
+    B_SB_FREE, B_P_READY, B_O_FULL, B_O_EMPTY, B_DS_FULL, B_DS_EMPTY, B_S_READY, B_SC_FULL0,
+    B_SC_FULL1, B_SC_FULL2, B_SC_FULL3, B_SC_EMPTY0, B_SC_EMPTY1, B_SC_EMPTY2, B_SC_EMPTY3,
+    B_ITEM_FULL0, B_ITEM_FULL1, B_ITEM_EMPTY0, B_ITEM_EMPTY1, B_FIN, B_CV_SYNC, B_PE_SYNC,
+    B_OS_SYNC, NUM_BARS
 };
 
 // tcgen05 instruction descriptors (kind::f16): D fp32, M = N = 128.
@@ -102,7 +105,7 @@ constexpr uint32_t idesc(uint32_t fmt, uint32_t a_mn_major, uint32_t b_mn_major)
            ((128u >> 3) << 17) | ((128u >> 4) << 24);
 }
 constexpr uint32_t F16 = 0, BF16 = 1;
-constexpr uint32_t IDESC_QK = idesc(BF16, 0, 0);  // Q K^T: bf16, both K-major
+constexpr uint32_t IDESC_QK = idesc(F16, 0, 0);   // Q K^T: both K-major
 constexpr uint32_t IDESC_PV = idesc(F16, 0, 1);   // P (TMEM) V: V MN-major
 constexpr uint32_t IDESC_QS = idesc(F16, 0, 0);   // Q S: S stored as rows of S^T (K-major)
 constexpr uint32_t IDESC_VK = idesc(F16, 1, 1);   // V^T Kt: both MN-major
@@ -119,7 +122,6 @@ struct Params {
     int num_items_dense;
     const float* slopes;
     void* o;
-    int out_f32;
     float* state_out;
     int reverse;
     WsHeader* hdr;
@@ -497,23 +499,54 @@ __device__ Item make_item(const Params& p, int t, int num_items)
 
 // ------------------------------------------------------------------ roles
 
+// Scales of one loaded block, handed from the converter group to the OS group
+// through a ring of four slots (B_SC_FULL / B_SC_EMPTY). Each byte is the
+// biased fp32 exponent of the factor that undoes a power-of-two scaling.
+struct ScaleRec {
+    uint8_t qe[C];  // Q rows (phase-C blocks)
+    uint8_t kc;     // K tile (phase C: K as fed to Q K^T; phase A: decayed keys)
+    uint8_t vc;     // V tile
+    uint8_t pad[14];
+};
+
 struct Smem {
     uint8_t* tiles;  // 1024-aligned: stage0 {Q,K,V}, stage1 {Q,K,V}, S16
     uint64_t* bars;
     Item* ring;
     volatile int* abort;
-    float* pw_pk;  // [C+1] lam^m of the PK group's current item
-    uint8_t* vs;   // [2][128] V row scales (biased exponents, by phase-C block parity)
-    uint8_t* pg;   // [2][128] P row scales
-    uint8_t* qe;   // [2][128] Q row scales
-    uint8_t* hs;   // [2][128] state-copy column scales
-    float* km;     // [2] decayed-key tile scales (slot ring, B_KM_FULL/EMPTY)
-    float* red;    // [2][4] partial maxima of the key-tile reduction
+    float* pw_pe;    // [C+1] lam^m of the PE group's current item
+    ScaleRec* sc;    // [4]
+    float* red;      // [2][8] partial tile maxima of the converter group
+    uint8_t* hs;     // [2][128] state-copy column scales (OS group)
     __device__ uint8_t* q(int s) const { return tiles + s * STAGE_BYTES; }
     __device__ uint8_t* k(int s) const { return tiles + s * STAGE_BYTES + TILE_BYTES; }
     __device__ uint8_t* v(int s) const { return tiles + s * STAGE_BYTES + 2 * TILE_BYTES; }
     __device__ uint8_t* s16() const { return tiles + 2 * STAGE_BYTES; }
 };
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int x, int y, int z, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)),
+        "l"(policy)
+        : "memory");
+}
 
 __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUtensorMap* tk,
                               const CUtensorMap* tv, const Smem& sm)
@@ -521,6 +554,9 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
     uint64_t* bars = sm.bars;
     const int num_items =
         p.cu_seqlens ? *reinterpret_cast<volatile int*>(&p.hdr->num_items) : p.num_items_dense;
+    // K and V read in phase A are read again in phase C: keep them in L2;
+    // everything read for the last time goes first.
+    const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
     uint32_t n_load = 0;
     uint32_t uses[2] = {0, 0};
     for (uint32_t k = 0;; ++k) {
@@ -534,37 +570,26 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
-        if (has_succ) {
-            for (int b = 0; b < nb && ok; ++b) {
+        for (int pass = has_succ ? 0 : 1; pass < 2 && ok; ++pass) {
+            for (int kb = 0; kb < nb; ++kb) {
                 const int s = n_load & 1;
                 ok = mbar_wait(&bars[B_EMPTY0 + s], ((n_load >> 1) & 1) ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
                 uint64_t* full = &bars[B_FULL0 + s];
-                mbar_expect_tx(full, 2 * TILE_BYTES);
-                const int y = it.y0 + block_t0(it.len, b, p.reverse);
-                tma_load_3d(sm.k(s), tk, full, 0, y, it.z);
-                tma_load_3d(sm.k(s) + BOX_BYTES, tk, full, 64, y, it.z);
-                tma_load_3d(sm.v(s), tv, full, 0, y, it.z);
-                tma_load_3d(sm.v(s) + BOX_BYTES, tv, full, 64, y, it.z);
+                const int y = it.y0 + block_t0(it.len, kb, p.reverse);
+                const uint64_t kv_pol = pass == 0 ? keep : drop;
+                mbar_expect_tx(full, (pass == 0 ? 2 : 3) * TILE_BYTES);
+                if (pass == 1) {
+                    tma_load_3d_hint(sm.q(s), tq, full, 0, y, it.z, drop);
+                    tma_load_3d_hint(sm.q(s) + BOX_BYTES, tq, full, 64, y, it.z, drop);
+                }
+                tma_load_3d_hint(sm.k(s), tk, full, 0, y, it.z, kv_pol);
+                tma_load_3d_hint(sm.k(s) + BOX_BYTES, tk, full, 64, y, it.z, kv_pol);
+                tma_load_3d_hint(sm.v(s), tv, full, 0, y, it.z, kv_pol);
+                tma_load_3d_hint(sm.v(s) + BOX_BYTES, tv, full, 64, y, it.z, kv_pol);
                 ++uses[s];
                 ++n_load;
             }
-        }
-        for (int kb = 0; kb < nb && ok; ++kb) {
-            const int s = n_load & 1;
-            ok = mbar_wait(&bars[B_EMPTY0 + s], ((n_load >> 1) & 1) ^ 1, sm.abort, p.hdr);
-            if (!ok) break;
-            uint64_t* full = &bars[B_FULL0 + s];
-            mbar_expect_tx(full, 3 * TILE_BYTES);
-            const int y = it.y0 + block_t0(it.len, kb, p.reverse);
-            tma_load_3d(sm.q(s), tq, full, 0, y, it.z);
-            tma_load_3d(sm.q(s) + BOX_BYTES, tq, full, 64, y, it.z);
-            tma_load_3d(sm.k(s), tk, full, 0, y, it.z);
-            tma_load_3d(sm.k(s) + BOX_BYTES, tk, full, 64, y, it.z);
-            tma_load_3d(sm.v(s), tv, full, 0, y, it.z);
-            tma_load_3d(sm.v(s) + BOX_BYTES, tv, full, 64, y, it.z);
-            ++uses[s];
-            ++n_load;
         }
         if (!ok) break;
     }
@@ -582,7 +607,8 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
 {
     uint64_t* bars = sm.bars;
     const uint32_t s16 = smem_u32(sm.s16());
-    uint32_t n_load = 0, n_kt[2] = {0, 0}, n_p = 0, n_q = 0, n_c1 = 0, n_o = 0, n_s = 0, n_ds = 0;
+    uint32_t n_load = 0, n_conv[2] = {0, 0}, n_kt[2] = {0, 0}, n_p = 0, n_c1 = 0, n_o = 0;
+    uint32_t n_s = 0, n_ds = 0;
     // DS^T = V^T Kt for the block in stage s (fresh accumulator), then release the stage.
     auto issue_vk = [&](int s) -> bool {
         if (!mbar_wait(&bars[B_KT0 + s], n_kt[s]++ & 1, sm.abort, p.hdr)) return false;
@@ -597,10 +623,10 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
         mma_commit(&bars[B_EMPTY0 + s]);
         return true;
     };
-    // SB = Q K^T for the block in stage (nl & 1).
+    // SB = Q K^T for the block in stage (nl & 1), once the converters are done with it.
     auto issue_qk = [&](uint32_t nl) -> bool {
         const int s = nl & 1;
-        if (!mbar_wait(&bars[B_FULL0 + s], (nl >> 1) & 1, sm.abort, p.hdr)) return false;
+        if (!mbar_wait(&bars[B_CONV0 + s], n_conv[s]++ & 1, sm.abort, p.hdr)) return false;
         if (!mbar_wait(&bars[B_SB_FREE], (n_c1++ & 1) ^ 1, sm.abort, p.hdr)) return false;
         tc_fence_after();
         const uint32_t qq = smem_u32(sm.q(s)), kk = smem_u32(sm.k(s));
@@ -642,8 +668,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
                 mma_ts(tmem + COL_OI, tmem + COL_SB + ks * 8, desc_mnmajor(vv, ks), IDESC_PV,
                        ks > 0 ? 1u : 0u);
             mma_commit(&bars[B_SB_FREE]);
-            ok = mbar_wait(&bars[B_Q_READY], n_q++ & 1, sm.abort, p.hdr) &&
-                 mbar_wait(&bars[B_S_READY], n_s++ & 1, sm.abort, p.hdr);
+            ok = mbar_wait(&bars[B_S_READY], n_s++ & 1, sm.abort, p.hdr);
             if (!ok) break;
             tc_fence_after();
 #pragma unroll
@@ -663,42 +688,96 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
     mbar_wait(&bars[B_FIN], 0, &never, p.hdr, DRAIN_LIMIT_NS);
 }
 
-__device__ void pk_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
+// Row r of a 16-bit tile as 64 packed words (two elements each).
+__device__ __forceinline__ void load_row_packed(const uint8_t* tile, int r, uint32_t (&w)[64])
+{
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const uint4 x = *reinterpret_cast<const uint4*>(tile + chunk_off(r, c));
+        w[4 * c + 0] = x.x;
+        w[4 * c + 1] = x.y;
+        w[4 * c + 2] = x.z;
+        w[4 * c + 3] = x.w;
+    }
+}
+
+__device__ __forceinline__ float absmax_bf16_packed(const uint32_t (&w)[64])
+{
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
+    return m;
+}
+
+// Store packed bf16 words times f as fp16 into row r.
+__device__ __forceinline__ void store_bf16_packed_as_f16(uint8_t* tile, int r,
+                                                         const uint32_t (&w)[64], float f)
+{
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        uint4 x;
+        x.x = pack_f16x2(bf16_lo(w[4 * c + 0]) * f, bf16_hi(w[4 * c + 0]) * f);
+        x.y = pack_f16x2(bf16_lo(w[4 * c + 1]) * f, bf16_hi(w[4 * c + 1]) * f);
+        x.z = pack_f16x2(bf16_lo(w[4 * c + 2]) * f, bf16_hi(w[4 * c + 2]) * f);
+        x.w = pack_f16x2(bf16_lo(w[4 * c + 3]) * f, bf16_hi(w[4 * c + 3]) * f);
+        *reinterpret_cast<uint4*>(tile + chunk_off(r, c)) = x;
+    }
+}
+
+// Max |x| of row r of a bf16 tile (streaming, few registers).
+__device__ __forceinline__ float row_absmax_bf16(const uint8_t* tile, int r)
+{
+    float m = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+        const uint4 x = *reinterpret_cast<const uint4*>(tile + chunk_off(r, c));
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(x.x)), fabsf(bf16_hi(x.x))),
+                           fmaxf(fabsf(bf16_lo(x.y)), fabsf(bf16_hi(x.y)))));
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(x.z)), fabsf(bf16_hi(x.z))),
+                           fmaxf(fabsf(bf16_lo(x.w)), fabsf(bf16_hi(x.w)))));
+    }
+    return m;
+}
+
+// Rewrite row r of a bf16 tile in place as fp16 times f (streaming).
+__device__ __forceinline__ void row_bf16_to_f16(uint8_t* tile, int r, float f)
+{
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+        uint4* ptr = reinterpret_cast<uint4*>(tile + chunk_off(r, c));
+        const uint4 x = *ptr;
+        *ptr = make_uint4(pack_f16x2(bf16_lo(x.x) * f, bf16_hi(x.x) * f),
+                          pack_f16x2(bf16_lo(x.y) * f, bf16_hi(x.y) * f),
+                          pack_f16x2(bf16_lo(x.z) * f, bf16_hi(x.z) * f),
+                          pack_f16x2(bf16_lo(x.w) * f, bf16_hi(x.w) * f));
+    }
+}
+
+// Converter group: fp16 operands for the tensor cores as soon as a block's
+// tiles land. Thread r owns row r of each tile. Q rows get their own
+// power-of-two scale; K and V get one scale per tile (a maximum over the
+// group). Phase-A blocks only need the decayed keys and V. The scales go to
+// the OS group through the ScaleRec ring.
+__device__ void cv_role(const Params& p, const Smem& sm, int warp, int lane)
 {
     uint64_t* bars = sm.bars;
-    const int row = ((warp & 3) << 5) | lane;  // TMEM lane == tile row
-    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) << 5) << 16);
+    const int r = ((warp & 3) << 5) | lane;
+    const int w = warp & 3;
     const int rev = p.reverse;
-    float* pw = sm.pw_pk;
-    uint32_t n_load = 0, n_sblk = 0, n_sync = 0, n_blk = 0, n_ds = 0;
+    uint32_t n_load = 0, n_sync = 0;
 
-    // Decayed keys of one block in stage s: Kt_j = k_j lam^(e_j) vup_j (zero
-    // beyond L), where vup_j undoes V row j's scale, then one power-of-two
-    // scale for the whole tile (max over the 128 rows, reduced through
-    // shared memory). The undo factor goes to km[] for the OS group.
-    auto make_kt = [&](int s, int L, float vup) -> bool {
-        float x[128];
-        load_row_bf16(sm.k(s), row, x);
-        const float f = row < L ? pw[rev ? row : L - 1 - row] * vup : 0.f;
-        float m = row_absmax(x) * f;
-        m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
-        float* red = sm.red + (n_ds & 1) * 4;
-        if (lane == 0) red[warp & 3] = m;
-        if (!group_sync(&bars[B_PK_SYNC], n_sync, sm.abort, p.hdr)) return false;
-        m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-        const Pow2 sc = pow2_for(m);
-        store_row_f16(sm.k(s), row, x, f * sc.down);
-        fence_proxy_async();
-        mbar_arrive(&bars[B_KT0 + s]);
-        if (row == 0) {
-            // Hand the tile's undo factor to the OS group (slot ring of two).
-            const int slot = n_ds & 1;
-            if (!mbar_wait(&bars[B_KM_EMPTY0 + slot], ((n_ds >> 1) & 1) ^ 1, sm.abort, p.hdr))
-                return false;
-            sm.km[slot] = sc.up;
-            mbar_arrive(&bars[B_KM_FULL0 + slot]);
+    // Tile maxima of (a, b) over the 128 rows.
+    auto tile_max2 = [&](float& a, float& b) -> bool {
+        a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a)));
+        b = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(b)));
+        float* red = sm.red + (n_load & 1) * 8;
+        if (lane == 0) {
+            red[w] = a;
+            red[4 + w] = b;
         }
-        ++n_ds;
+        if (!group_sync(&bars[B_CV_SYNC], n_sync, sm.abort, p.hdr)) return false;
+        a = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+        b = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
         return true;
     };
 
@@ -710,112 +789,154 @@ __device__ void pk_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         if (lane == 0) mbar_arrive(&bars[B_ITEM_EMPTY0 + slot]);
         if (!it.valid) break;
         const float slope = p.slopes[it.head];
-        if (!group_sync(&bars[B_PK_SYNC], n_sync, sm.abort, p.hdr)) break;
-        pw[row] = expf(-slope * (float)row);
-        if (row == 0) pw[C] = expf(-slope * (float)C);
-        if (!group_sync(&bars[B_PK_SYNC], n_sync, sm.abort, p.hdr)) break;
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
-        if (has_succ) {
-            // Phase A: V conversion and decayed keys only.
+        for (int pass = has_succ ? 0 : 1; pass < 2 && ok; ++pass) {
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int s = n_load & 1;
                 const int L = min(C, it.len - block_t0(it.len, kb, rev));
-                ok = wait_warp(&bars[B_FULL0 + s], (n_load >> 1) & 1, sm.abort, p.hdr);
+                const int sl = n_load & 3;
+                ScaleRec* rec = sm.sc + sl;
+                ok = wait_warp(&bars[B_FULL0 + s], (n_load >> 1) & 1, sm.abort, p.hdr) &&
+                     wait_warp(&bars[B_SC_EMPTY0 + sl], ((n_load >> 2) & 1) ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
-                ok = make_kt(s, L, convert_row(sm.v(s), row, L).up);
+                const bool live = r < L;
+                if (pass == 1) {
+                    // Q: own scale per row.
+                    const Pow2 qs = pow2_for(row_absmax_bf16(sm.q(s), r));
+                    row_bf16_to_f16(sm.q(s), r, qs.down);
+                    rec->qe[r] = qs.ue;
+                }
+                // K (phase A: already decayed) and V: one scale per tile.
+                const float kf = pass == 0
+                                     ? (live ? expf(-slope * (float)(rev ? r : L - 1 - r)) : 0.f)
+                                     : (live ? 1.f : 0.f);
+                float km = row_absmax_bf16(sm.k(s), r) * kf;
+                float vm = live ? row_absmax_bf16(sm.v(s), r) : 0.f;
+                if (!(ok = tile_max2(km, vm))) break;
+                const Pow2 ks = pow2_for(km), vs = pow2_for(vm);
+                row_bf16_to_f16(sm.k(s), r, kf * ks.down);
+                row_bf16_to_f16(sm.v(s), r, live ? vs.down : 0.f);
+                if (r == 0) {
+                    rec->kc = ks.ue;
+                    rec->vc = vs.ue;
+                }
+                fence_proxy_async();
+                mbar_arrive(&bars[pass == 0 ? B_KT0 + s : B_CONV0 + s]);
+                mbar_arrive(&bars[B_SC_FULL0 + sl]);
                 ++n_load;
             }
         }
+        if (!ok) break;
+    }
+}
+
+// PE group: after Q K^T, the decayed causal mask (fp16 P into TMEM, in place
+// over the scores) and the decayed keys for the state update (in place over
+// K). Thread i owns TMEM lane / tile row i.
+template <int REV>
+__device__ void pe_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
+{
+    uint64_t* bars = sm.bars;
+    const int w = warp & 3;
+    const int row = (w << 5) | lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(w << 5) << 16);
+    float* pw = sm.pw_pe;
+    uint32_t n_load = 0, n_sblk = 0, n_sync = 0;
+    for (uint32_t k = 0;; ++k) {
+        const int slot = k & 1;
+        if (!wait_warp(&bars[B_ITEM_FULL0 + slot], (k >> 1) & 1, sm.abort, p.hdr)) break;
+        const Item it = sm.ring[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_ITEM_EMPTY0 + slot]);
+        if (!it.valid) break;
+        const float slope = p.slopes[it.head];
+        if (!group_sync(&bars[B_PE_SYNC], n_sync, sm.abort, p.hdr)) break;
+        pw[row] = expf(-slope * (float)row);
+        if (row == 0) pw[C] = expf(-slope * (float)C);
+        if (!group_sync(&bars[B_PE_SYNC], n_sync, sm.abort, p.hdr)) break;
+        const int nb = num_blocks(it.len);
+        if (it.p_ord < it.nseg - 1) n_load += nb;  // phase A blocks need no PE work
+        bool ok = true;
         for (int kb = 0; kb < nb && ok; ++kb) {
             const int s = n_load & 1;
-            const int par = n_blk & 1;
-            const int L = min(C, it.len - block_t0(it.len, kb, rev));
-            // V -> fp16 (row scales to vs[] for E_P).
-            ok = wait_warp(&bars[B_FULL0 + s], (n_load >> 1) & 1, sm.abort, p.hdr);
+            const int L = min(C, it.len - block_t0(it.len, kb, REV));
+            ok = wait_warp(&bars[B_SBLK_FULL], n_sblk++ & 1, sm.abort, p.hdr);
             if (!ok) break;
-            const Pow2 vsc = convert_row(sm.v(s), row, L);
-            const float vup = vsc.up;
-            sm.vs[par * C + row] = vsc.ue;
-            fence_proxy_async();
-            if (!(ok = group_sync(&bars[B_PK_SYNC], n_sync, sm.abort, p.hdr))) break;
-            // E_P: decayed causal mask times V's row scales, row-normalized, fp16 into TMEM.
-            if (!(ok = wait_warp(&bars[B_SBLK_FULL], n_sblk++ & 1, sm.abort, p.hdr))) break;
             tc_fence_after();
-            {
-                // Two passes over SB: the row maximum, then scaled fp16 P (the
-                // second pass writes P into columns it has already read).
-                const uint8_t* vsp = sm.vs + par * C;
-                float mx = 0.f;
+            // E_P. Chunk c covers columns 32c..32c+31; warp w holds rows
+            // 32w..32w+31, so chunks before (forward) / after (reverse) the
+            // diagonal chunk are fully causal and the rest fully masked.
+            const bool row_live = REV ? true : row < L;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(lane_addr + COL_SB + 32 * c, r);
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+                const bool active = REV ? (c >= w) : (c <= w);
+                if (active) {
+                    uint32_t r32[32];
+                    tmem_ld32(lane_addr + COL_SB + 32 * c, r32);
                     tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = 32 * c + e;
-                        const bool keep = rev ? (j >= row && j < L) : (j <= row && row < L);
-                        const int m = keep ? (rev ? j - row : row - j) : 0;
-                        const float x = keep ? __uint_as_float(r[e]) * pw[m] * up_of(vsp[j]) : 0.f;
-                        mx = fmaxf(mx, fabsf(x));
-                    }
-                }
-                const Pow2 sc = pow2_for(mx);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32(lane_addr + COL_SB + 32 * c, r);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         float x2[2];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const int j = 32 * c + e + u;
-                            const bool keep = rev ? (j >= row && j < L) : (j <= row && row < L);
-                            const int m = keep ? (rev ? j - row : row - j) : 0;
-                            x2[u] = keep ? __uint_as_float(r[e + u]) * pw[m] * up_of(vsp[j]) * sc.down
-                                         : 0.f;
+                            bool keep;
+                            int m;
+                            if (REV) {
+                                keep = (c > w || j >= row) && j < L;
+                                m = j - row;
+                            } else {
+                                keep = (c < w || j <= row) && row_live;
+                                m = row - j;
+                            }
+                            x2[u] = keep ? __uint_as_float(r32[e + u]) * pw[keep ? m : 0] : 0.f;
                         }
                         pk[e >> 1] = pack_f16x2(x2[0], x2[1]);
                     }
-                    tmem_st16(lane_addr + COL_SB + 16 * c, pk);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
                 }
-                sm.pg[par * C + row] = sc.ue;
+                tmem_st16(lane_addr + COL_SB + 16 * c, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars[B_P_READY]);
-            // Q -> fp16 for MMA3 (row scales to qe[] for E_O).
-            sm.qe[par * C + row] = convert_row(sm.q(s), row, C).ue;
+            // E_K: decayed keys lam^(L-1-j) k_j (reverse: lam^j), in place (fp16).
+            {
+                const float f = row < L ? pw[REV ? row : L - 1 - row] : 0.f;
+                uint8_t* kt = sm.k(s);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    uint4* ptr = reinterpret_cast<uint4*>(kt + chunk_off(row, c));
+                    uint4 x = *ptr;
+                    uint32_t* e4 = reinterpret_cast<uint32_t*>(&x);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&e4[u]));
+                        e4[u] = pack_f16x2(h.x * f, h.y * f);
+                    }
+                    *ptr = x;
+                }
+            }
             fence_proxy_async();
-            mbar_arrive(&bars[B_Q_READY]);
-            // E_K.
-            ok = make_kt(s, L, vup);
+            mbar_arrive(&bars[B_KT0 + s]);
             ++n_load;
-            ++n_blk;
         }
         if (!ok) break;
     }
 }
 
-// OS group: S = lam^L S + up_K * DS for the next DS use. Waits for the MMA
-// and for the key-tile scale, then frees DS and the scale slot.
-// n_ds counts DS uses so far.
+// OS group: S = lam^L S + up * DS for the next DS use (phase A or C).
 __device__ __forceinline__ bool os_accumulate_ds(const Params& p, const Smem& sm,
                                                  uint32_t lane_addr, float (&S)[D], int L,
-                                                 float slope, uint32_t& n_ds)
+                                                 float slope, float up, uint32_t& n_ds)
 {
-    const int slot = n_ds & 1;
     if (!wait_warp(&sm.bars[B_DS_FULL], n_ds & 1, sm.abort, p.hdr)) return false;
-    if (!wait_warp(&sm.bars[B_KM_FULL0 + slot], (n_ds >> 1) & 1, sm.abort, p.hdr)) return false;
     tc_fence_after();
-    const float up = sm.km[slot];
-    mbar_arrive(&sm.bars[B_KM_EMPTY0 + slot]);
-    ++n_ds;
     const float dL = expf(-slope * (float)L);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -828,6 +949,8 @@ __device__ __forceinline__ bool os_accumulate_ds(const Params& p, const Smem& sm
     }
     tc_fence_before();
     mbar_arrive(&sm.bars[B_DS_EMPTY]);
+    mbar_arrive(&sm.bars[B_SC_EMPTY0 + (n_ds & 3)]);
+    ++n_ds;
     return true;
 }
 
@@ -841,15 +964,15 @@ __device__ __forceinline__ void os_publish_s16(const Smem& sm, int a, const floa
     mbar_arrive(&sm.bars[B_S_READY]);
 }
 
+template <int REV, int OUT_F32>
 __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
     uint64_t* bars = sm.bars;
     const int a = ((warp & 3) << 5) | lane;  // TMEM lane: output row i / state column a
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) << 5) << 16);
-    const int rev = p.reverse;
     float slope = 0.f;
-    // n_blk counts phase-C blocks (one o_full, q_ready and s_ready phase each);
-    // n_ds counts DS uses (= blocks loaded).
+    // n_blk counts phase-C blocks (one o_full and s_ready phase each);
+    // n_ds counts DS uses (= blocks loaded = scale records).
     uint32_t n_sync = 0, n_blk = 0, n_ds = 0;
     float S[D];  // column a of the fp32 state: S[x] = state[x][a]
 
@@ -870,8 +993,12 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         if (has_succ) {
             // Phase A: local state of the segment.
             for (int kb = 0; kb < nb && ok; ++kb) {
-                const int L = min(C, it.len - block_t0(it.len, kb, rev));
-                ok = os_accumulate_ds(p, sm, lane_addr, S, L, slope, n_ds);
+                const int L = min(C, it.len - block_t0(it.len, kb, REV));
+                const ScaleRec* rec = sm.sc + (n_ds & 3);
+                ok = wait_warp(&bars[B_SC_FULL0 + (n_ds & 3)], (n_ds >> 2) & 1, sm.abort, p.hdr);
+                if (!ok) break;
+                const float up = up_of(rec->kc) * up_of(rec->vc);
+                ok = os_accumulate_ds(p, sm, lane_addr, S, L, slope, up, n_ds);
             }
             if (!ok) break;
         }
@@ -930,17 +1057,20 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
 
         for (int kb = 0; kb < nb && ok; ++kb) {
             const int par = n_blk & 1;
-            const int t0 = block_t0(it.len, kb, rev);
+            const int t0 = block_t0(it.len, kb, REV);
             const int L = min(C, it.len - t0);
-            // E_O: O = up_P * OI + lam^(i+1) * up_Q * up_S[col] * OE (reverse: lam^(L-i)).
+            const ScaleRec* rec = sm.sc + (n_ds & 3);
+            // E_O: O = up_Q up_K up_V * OI + lam^(i+1) * up_Q * up_S[col] * OE
+            // (reverse: lam^(L-i)).
             ok = wait_warp(&bars[B_O_FULL], n_blk & 1, sm.abort, p.hdr) &&
-                 wait_warp(&bars[B_Q_READY], n_blk & 1, sm.abort, p.hdr) &&
-                 wait_warp(&bars[B_S_READY], n_blk & 1, sm.abort, p.hdr);
+                 wait_warp(&bars[B_S_READY], n_blk & 1, sm.abort, p.hdr) &&
+                 wait_warp(&bars[B_SC_FULL0 + (n_ds & 3)], (n_ds >> 2) & 1, sm.abort, p.hdr);
             if (!ok) break;
             tc_fence_after();
-            const float gi = up_of(sm.pg[par * C + a]);
-            const float rowc = expf(-slope * (float)(rev ? max(L - a, 0) : a + 1)) *
-                               up_of(sm.qe[par * C + a]);
+            const float up_kv = up_of(rec->kc) * up_of(rec->vc);
+            const float up_q = up_of(rec->qe[a]);
+            const float gi = up_q * up_kv;
+            const float rowc = expf(-slope * (float)(REV ? max(L - a, 0) : a + 1)) * up_q;
             const uint8_t* hsp = sm.hs + par * C;
             const bool store = a < L;
             const long long orow = it.out_row0 + t0 + a;
@@ -956,7 +1086,7 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
                     ov[x] = fmaf(rowc * up_of(hsp[8 * c + x]), __uint_as_float(re[x]),
                                  gi * __uint_as_float(ri[x]));
                 if (store) {
-                    if (p.out_f32) {
+                    if (OUT_F32) {
                         float4* dst = reinterpret_cast<float4*>(
                             static_cast<float*>(p.o) + orow * D + 8 * c);
                         dst[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
@@ -972,7 +1102,7 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
             tc_fence_before();
             mbar_arrive(&bars[B_O_EMPTY]);
             // E_S.
-            if (!(ok = os_accumulate_ds(p, sm, lane_addr, S, L, slope, n_ds))) break;
+            if (!(ok = os_accumulate_ds(p, sm, lane_addr, S, L, slope, up_kv, n_ds))) break;
             if (kb + 1 < nb) os_publish_s16(sm, a, S, (n_blk + 1) & 1);
             ++n_blk;
         }
@@ -990,18 +1120,20 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
 constexpr uint32_t SM_BARS = 0;                       // 32 x 8 B
 constexpr uint32_t SM_RING = 256;                     // 2 x Item
 constexpr uint32_t SM_PW = 384;                       // (C+1) floats
-constexpr uint32_t SM_SCALES = 912;                   // 4 x [2][128] bytes
-constexpr uint32_t SM_KM = SM_SCALES + 1024;          // 4 floats
-constexpr uint32_t SM_RED = SM_KM + 16;               // 8 floats
-constexpr uint32_t SM_TMEM = SM_RED + 32;             // u32
+constexpr uint32_t SM_SC = 912;                       // 4 x ScaleRec (144 B)
+constexpr uint32_t SM_RED = SM_SC + 4 * 144;          // 16 floats
+constexpr uint32_t SM_HS = SM_RED + 64;               // [2][128] bytes
+constexpr uint32_t SM_TMEM = SM_HS + 256;             // u32
 constexpr uint32_t SM_ABORT = SM_TMEM + 4;            // int
 constexpr uint32_t SM_SMALL = SM_ABORT + 4;
 static_assert(NUM_BARS <= 32, "barrier area");
 static_assert(sizeof(Item) * 2 <= SM_PW - SM_RING, "ring area");
-static_assert(SM_PW + (C + 1) * 4 <= SM_SCALES, "pw area");
+static_assert(SM_PW + (C + 1) * 4 <= SM_SC, "pw area");
+static_assert(sizeof(ScaleRec) == 144, "scale record");
 constexpr uint32_t SMEM_BYTES = SM_SMALL + 1023 + SMEM_TILES;
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
+template <int REV, int OUT_F32>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_forward_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv, const Params p)
@@ -1017,22 +1149,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     sm.bars = bars;
     sm.ring = reinterpret_cast<Item*>(dsmem + SM_RING);
     sm.abort = abort_flag;
-    sm.pw_pk = reinterpret_cast<float*>(dsmem + SM_PW);
-    sm.vs = dsmem + SM_SCALES;
-    sm.pg = dsmem + SM_SCALES + 256;
-    sm.qe = dsmem + SM_SCALES + 512;
-    sm.hs = dsmem + SM_SCALES + 768;
-    sm.km = reinterpret_cast<float*>(dsmem + SM_KM);
+    sm.pw_pe = reinterpret_cast<float*>(dsmem + SM_PW);
+    sm.sc = reinterpret_cast<ScaleRec*>(dsmem + SM_SC);
     sm.red = reinterpret_cast<float*>(dsmem + SM_RED);
+    sm.hs = dsmem + SM_HS;
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
         uint32_t counts[NUM_BARS];
-        for (int i = 0; i < NUM_BARS; ++i) counts[i] = 1;
-        counts[B_KT0] = counts[B_KT1] = counts[B_P_READY] = counts[B_O_EMPTY] = 128;
-        counts[B_DS_EMPTY] = counts[B_S_READY] = counts[B_PK_SYNC] = counts[B_OS_SYNC] = 128;
-        counts[B_Q_READY] = counts[B_KM_EMPTY0] = counts[B_KM_EMPTY1] = 128;
-        counts[B_ITEM_EMPTY0] = counts[B_ITEM_EMPTY1] = 9;  // MMA lane + 4 + 4 epilogue warps
+        for (int i = 0; i < NUM_BARS; ++i) counts[i] = 128;
+        counts[B_FULL0] = counts[B_FULL1] = counts[B_EMPTY0] = counts[B_EMPTY1] = 1;
+        counts[B_SBLK_FULL] = counts[B_SB_FREE] = counts[B_O_FULL] = counts[B_DS_FULL] = 1;
+        counts[B_ITEM_FULL0] = counts[B_ITEM_FULL1] = counts[B_FIN] = 1;
+        counts[B_ITEM_EMPTY0] = counts[B_ITEM_EMPTY1] = 13;  // MMA lane + 12 group warps
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], counts[i]);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tq)) : "memory");
@@ -1055,10 +1184,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (warp == 0 && lane == 0) producer_role(p, &tq, &tk, &tv, sm);
         if (warp == 1 && lane == 0) mma_role(p, sm, tmem);
     } else if (warp < 8) {
-        pk_role(p, sm, tmem, warp, lane);
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_CV));
+        cv_role(p, sm, warp, lane);
+    } else if (warp < 12) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PE));
+        pe_role<REV>(p, sm, tmem, warp, lane);
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_OS));
-        os_role(p, sm, tmem, warp, lane);
+        os_role<REV, OUT_F32>(p, sm, tmem, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -1267,7 +1400,6 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     prm.num_items_dense = varlen ? 0 : (int)w.max_items;
     prm.slopes = slopes;
     prm.o = o;
-    prm.out_f32 = out_t == LA_F32;
     prm.state_out = state_out;
     prm.reverse = reverse;
     prm.hdr = reinterpret_cast<WsHeader*>(ws);
@@ -1289,18 +1421,20 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         if (P.total == 0) return cudaSuccess;
     }
-    static bool attr_done = false;
-    if (!attr_done) {
-        err = cudaFuncSetAttribute(tc_forward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)SMEM_BYTES);
-        if (err != cudaSuccess) return err;
-        attr_done = true;
-    }
     const long long max_items = w.max_items;
     const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(1, max_items));
-    tc_forward_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
-    count_launch();
-    return cudaGetLastError();
+    auto launch = [&](auto kern) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+        count_launch();
+        return cudaGetLastError();
+    };
+    const bool f32 = out_t == LA_F32;
+    if (reverse)
+        return f32 ? launch(tc_forward_kernel<1, 1>) : launch(tc_forward_kernel<1, 0>);
+    return f32 ? launch(tc_forward_kernel<0, 1>) : launch(tc_forward_kernel<0, 0>);
 }
 
 cudaError_t launch_tc_backward(const Problems& P, const void* dO, const void* q, const void* k,
