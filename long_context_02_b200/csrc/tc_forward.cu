@@ -47,9 +47,9 @@
 // epilogues.
 //
 // Warp roles (16 warps, 4 warpgroups): warp 0 TMA producer, warp 1 MMA
-// issuer (also owns TMEM), warps 2-3 idle; 4-7 converters (fp16 Q, K, V as
-// tiles land); 8-11 "PE" (E_P and E_K after Q K^T); 12-15 "OS" (E_O, E_S and
-// the scan). TMEM: 512 columns = SB/P | OI | OE | DS^T, 128 lanes.
+// issuer (also owns TMEM), warps 2-3 Q converters; 4-7 K/V converters (fp16
+// tiles as they land); 8-11 "PE" (E_P and E_K after Q K^T); 12-15 "OS" (E_O,
+// E_S and the scan). TMEM: 512 columns = SB/P | OI | OE | DS^T, 128 lanes.
 // Shared memory: 2 stages x (Q, K, V) 128x128 16-bit tiles + the fp16 state
 // copy, all in the 128-byte-swizzled layout TMA writes.
 //
@@ -92,8 +92,12 @@ enum {
     B_SB_FREE, B_P_READY, B_O_FULL, B_O_EMPTY, B_DS_FULL, B_DS_EMPTY, B_S_READY, B_SC_FULL0,
     B_SC_FULL1, B_SC_FULL2, B_SC_FULL3, B_SC_EMPTY0, B_SC_EMPTY1, B_SC_EMPTY2, B_SC_EMPTY3,
     B_ITEM_FULL0, B_ITEM_FULL1, B_ITEM_EMPTY0, B_ITEM_EMPTY1, B_FIN, B_CV_SYNC, B_PE_SYNC,
-    B_OS_SYNC, NUM_BARS
+    B_OS_SYNC, B_QFULL0, B_QFULL1, NUM_BARS
 };
+// A barrier's waiter must not skip phases: a parity wait on a barrier two
+// phases behind returns at once. So the Q tile, which only phase-C blocks
+// load, completes its own B_QFULL barrier rather than B_FULL, which every
+// block completes and the Q converters would otherwise skip in phase A.
 
 // tcgen05 instruction descriptors (kind::f16): D fp32, M = N = 128.
 // bits: [4,6) D format (1 = f32), [7,10) A format and [10,13) B format
@@ -286,7 +290,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
           "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
           "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
           "=r"(r[31])
-        : "r"(taddr));
+        : "r"(taddr)
+        : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
@@ -297,7 +302,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
           "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
+        : "r"(taddr)
+        : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
@@ -305,7 +311,8 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                    "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr));
+                 : "r"(taddr)
+                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
@@ -517,7 +524,7 @@ struct Smem {
     float* pw_pe;    // [C+1] lam^m of the PE group's current item
     ScaleRec* sc;    // [4]
     float* red;      // [2][8] partial tile maxima of the converter group
-    uint8_t* hs;     // [2][128] state-copy column scales (OS group)
+    uint8_t* hs;     // [2][4] state-copy scales, one per 32 columns (OS group)
     __device__ uint8_t* q(int s) const { return tiles + s * STAGE_BYTES; }
     __device__ uint8_t* k(int s) const { return tiles + s * STAGE_BYTES + TILE_BYTES; }
     __device__ uint8_t* v(int s) const { return tiles + s * STAGE_BYTES + 2 * TILE_BYTES; }
@@ -558,7 +565,7 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
     // everything read for the last time goes first.
     const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
     uint32_t n_load = 0;
-    uint32_t uses[2] = {0, 0};
+    uint32_t uses[2] = {0, 0}, quses[2] = {0, 0};
     for (uint32_t k = 0;; ++k) {
         const int slot = k & 1;
         if (!mbar_wait(&bars[B_ITEM_EMPTY0 + slot], ((k >> 1) & 1) ^ 1, sm.abort, p.hdr)) break;
@@ -578,10 +585,13 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
                 uint64_t* full = &bars[B_FULL0 + s];
                 const int y = it.y0 + block_t0(it.len, kb, p.reverse);
                 const uint64_t kv_pol = pass == 0 ? keep : drop;
-                mbar_expect_tx(full, (pass == 0 ? 2 : 3) * TILE_BYTES);
+                mbar_expect_tx(full, 2 * TILE_BYTES);
                 if (pass == 1) {
-                    tma_load_3d_hint(sm.q(s), tq, full, 0, y, it.z, drop);
-                    tma_load_3d_hint(sm.q(s) + BOX_BYTES, tq, full, 64, y, it.z, drop);
+                    uint64_t* qfull = &bars[B_QFULL0 + s];
+                    mbar_expect_tx(qfull, TILE_BYTES);
+                    tma_load_3d_hint(sm.q(s), tq, qfull, 0, y, it.z, drop);
+                    tma_load_3d_hint(sm.q(s) + BOX_BYTES, tq, qfull, 64, y, it.z, drop);
+                    ++quses[s];
                 }
                 tma_load_3d_hint(sm.k(s), tk, full, 0, y, it.z, kv_pol);
                 tma_load_3d_hint(sm.k(s) + BOX_BYTES, tk, full, 64, y, it.z, kv_pol);
@@ -599,6 +609,9 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
             if (uses[s] > 0) {
                 volatile int never = 0;
                 mbar_wait(&bars[B_FULL0 + s], (uses[s] - 1) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
+                if (quses[s] > 0)
+                    mbar_wait(&bars[B_QFULL0 + s], (quses[s] - 1) & 1, &never, p.hdr,
+                              DRAIN_LIMIT_NS);
             }
     }
 }
@@ -676,8 +689,10 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
                 mma_ss(tmem + COL_OE, desc_kmajor(qq, ks), desc_kmajor(s16, ks), IDESC_QS,
                        ks > 0 ? 1u : 0u);
             mma_commit(&bars[B_O_FULL]);
-            if (kb + 1 < nb && !(ok = issue_qk(n_load + 1))) break;
+            // MMA4 of this block, then MMA1 of the next (its tiles are converted
+            // while this block's epilogues run).
             if (!(ok = issue_vk(s))) break;
+            if (kb + 1 < nb && !(ok = issue_qk(n_load + 1))) break;
             ++n_load;
         }
         if (!ok) break;
@@ -724,19 +739,19 @@ __device__ __forceinline__ void store_bf16_packed_as_f16(uint8_t* tile, int r,
     }
 }
 
-// Max |x| of row r of a bf16 tile (streaming, few registers).
+// Max |x| of row r of a bf16 tile (streaming, few registers). With the sign
+// bit cleared, bf16 bit patterns order like their magnitudes, so the maximum
+// is a packed unsigned 16-bit maximum.
 __device__ __forceinline__ float row_absmax_bf16(const uint8_t* tile, int r)
 {
-    float m = 0.f;
+    uint32_t m = 0u;
 #pragma unroll 4
     for (int c = 0; c < 16; ++c) {
         const uint4 x = *reinterpret_cast<const uint4*>(tile + chunk_off(r, c));
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(x.x)), fabsf(bf16_hi(x.x))),
-                           fmaxf(fabsf(bf16_lo(x.y)), fabsf(bf16_hi(x.y)))));
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(x.z)), fabsf(bf16_hi(x.z))),
-                           fmaxf(fabsf(bf16_lo(x.w)), fabsf(bf16_hi(x.w)))));
+        m = __vmaxu2(m, __vmaxu2(__vmaxu2(x.x & 0x7fff7fffu, x.y & 0x7fff7fffu),
+                                 __vmaxu2(x.z & 0x7fff7fffu, x.w & 0x7fff7fffu)));
     }
-    return m;
+    return fmaxf(bf16_lo(m), bf16_hi(m));
 }
 
 // Rewrite row r of a bf16 tile in place as fp16 times f (streaming).
@@ -750,6 +765,50 @@ __device__ __forceinline__ void row_bf16_to_f16(uint8_t* tile, int r, float f)
                           pack_f16x2(bf16_lo(x.y) * f, bf16_hi(x.y) * f),
                           pack_f16x2(bf16_lo(x.z) * f, bf16_hi(x.z) * f),
                           pack_f16x2(bf16_lo(x.w) * f, bf16_hi(x.w) * f));
+    }
+}
+
+// Q converters (the two spare warps of the control warpgroup): fp16 Q with
+// one power-of-two scale per row, for phase-C blocks, in parallel with the K
+// and V converters. Thread t owns rows t and t + 64.
+__device__ void qcv_role(const Params& p, const Smem& sm, int warp, int lane)
+{
+    uint64_t* bars = sm.bars;
+    const int t = ((warp & 1) << 5) | lane;
+    uint32_t n_load = 0, n_q[2] = {0, 0};
+    for (uint32_t k = 0;; ++k) {
+        const int slot = k & 1;
+        if (!wait_warp(&bars[B_ITEM_FULL0 + slot], (k >> 1) & 1, sm.abort, p.hdr)) break;
+        const Item it = sm.ring[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_ITEM_EMPTY0 + slot]);
+        if (!it.valid) break;
+        const int nb = num_blocks(it.len);
+        bool ok = true;
+        for (int pass = it.p_ord < it.nseg - 1 ? 0 : 1; pass < 2 && ok; ++pass) {
+            for (int kb = 0; kb < nb && ok; ++kb) {
+                const int s = n_load & 1;
+                const int sl = n_load & 3;
+                ok = wait_warp(&bars[B_SC_EMPTY0 + sl], ((n_load >> 2) & 1) ^ 1, sm.abort, p.hdr);
+                if (!ok) break;
+                if (pass == 1) {
+                    ok = wait_warp(&bars[B_QFULL0 + s], n_q[s]++ & 1, sm.abort, p.hdr);
+                    if (!ok) break;
+#pragma unroll 1
+                    for (int h = 0; h < 2; ++h) {
+                        const int r = t + 64 * h;
+                        const Pow2 qs = pow2_for(row_absmax_bf16(sm.q(s), r));
+                        row_bf16_to_f16(sm.q(s), r, qs.down);
+                        sm.sc[sl].qe[r] = qs.ue;
+                    }
+                    fence_proxy_async();
+                    mbar_arrive(&bars[B_CONV0 + s]);
+                }
+                mbar_arrive(&bars[B_SC_FULL0 + sl]);
+                ++n_load;
+            }
+        }
+        if (!ok) break;
     }
 }
 
@@ -802,12 +861,6 @@ __device__ void cv_role(const Params& p, const Smem& sm, int warp, int lane)
                      wait_warp(&bars[B_SC_EMPTY0 + sl], ((n_load >> 2) & 1) ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
                 const bool live = r < L;
-                if (pass == 1) {
-                    // Q: own scale per row.
-                    const Pow2 qs = pow2_for(row_absmax_bf16(sm.q(s), r));
-                    row_bf16_to_f16(sm.q(s), r, qs.down);
-                    rec->qe[r] = qs.ue;
-                }
                 // K (phase A: already decayed) and V: one scale per tile.
                 const float kf = pass == 0
                                      ? (live ? expf(-slope * (float)(rev ? r : L - 1 - r)) : 0.f)
@@ -816,8 +869,8 @@ __device__ void cv_role(const Params& p, const Smem& sm, int warp, int lane)
                 float vm = live ? row_absmax_bf16(sm.v(s), r) : 0.f;
                 if (!(ok = tile_max2(km, vm))) break;
                 const Pow2 ks = pow2_for(km), vs = pow2_for(vm);
-                row_bf16_to_f16(sm.k(s), r, kf * ks.down);
                 row_bf16_to_f16(sm.v(s), r, live ? vs.down : 0.f);
+                row_bf16_to_f16(sm.k(s), r, kf * ks.down);
                 if (r == 0) {
                     rec->kc = ks.ue;
                     rec->vc = vs.ue;
@@ -939,13 +992,13 @@ __device__ __forceinline__ bool os_accumulate_ds(const Params& p, const Smem& sm
     tc_fence_after();
     const float dL = expf(-slope * (float)L);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint32_t r[16];
-        tmem_ld16(lane_addr + COL_DS + 16 * c, r);
+    for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_addr + COL_DS + 32 * c, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 16; ++x)
-            S[16 * c + x] = fmaf(dL, S[16 * c + x], up * __uint_as_float(r[x]));
+        for (int x = 0; x < 32; ++x)
+            S[32 * c + x] = fmaf(dL, S[32 * c + x], up * __uint_as_float(r[x]));
     }
     tc_fence_before();
     mbar_arrive(&sm.bars[B_DS_EMPTY]);
@@ -954,12 +1007,14 @@ __device__ __forceinline__ bool os_accumulate_ds(const Params& p, const Smem& sm
     return true;
 }
 
-// OS group: fp16 copy of the state for MMA3 (row a of S^T, scaled per column).
+// OS group: fp16 copy of the state for MMA3 (row a of S^T). One power-of-two
+// scale per 32 state columns (one warp), from a warp-wide maximum.
 __device__ __forceinline__ void os_publish_s16(const Smem& sm, int a, const float (&S)[D], int par)
 {
-    const Pow2 sc = pow2_for(row_absmax(S));
+    const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(row_absmax(S))));
+    const Pow2 sc = pow2_for(m);
     store_row_f16(sm.s16(), a, S, sc.down);
-    sm.hs[par * C + a] = sc.ue;
+    if ((a & 31) == 0) sm.hs[par * 4 + (a >> 5)] = sc.ue;
     fence_proxy_async();
     mbar_arrive(&sm.bars[B_S_READY]);
 }
@@ -1071,31 +1126,34 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
             const float up_q = up_of(rec->qe[a]);
             const float gi = up_q * up_kv;
             const float rowc = expf(-slope * (float)(REV ? max(L - a, 0) : a + 1)) * up_q;
-            const uint8_t* hsp = sm.hs + par * C;
+            const uint8_t* hsp = sm.hs + par * 4;
             const bool store = a < L;
             const long long orow = it.out_row0 + t0 + a;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                uint32_t ri[8], re[8];
-                tmem_ld8(lane_addr + COL_OI + 8 * c, ri);
-                tmem_ld8(lane_addr + COL_OE + 8 * c, re);
+            for (int c = 0; c < 8; ++c) {
+                uint32_t ri[16], re[16];
+                tmem_ld16(lane_addr + COL_OI + 16 * c, ri);
+                tmem_ld16(lane_addr + COL_OE + 16 * c, re);
                 tmem_wait_ld();
-                float ov[8];
 #pragma unroll
-                for (int x = 0; x < 8; ++x)
-                    ov[x] = fmaf(rowc * up_of(hsp[8 * c + x]), __uint_as_float(re[x]),
-                                 gi * __uint_as_float(ri[x]));
-                if (store) {
-                    if (OUT_F32) {
-                        float4* dst = reinterpret_cast<float4*>(
-                            static_cast<float*>(p.o) + orow * D + 8 * c);
-                        dst[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
-                        dst[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
-                    } else {
-                        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow * D +
-                                                  8 * c) =
-                            make_uint4(pack_bf16x2(ov[0], ov[1]), pack_bf16x2(ov[2], ov[3]),
-                                       pack_bf16x2(ov[4], ov[5]), pack_bf16x2(ov[6], ov[7]));
+                for (int h = 0; h < 2; ++h) {
+                    float ov[8];
+                    const float ec = rowc * up_of(hsp[c >> 1]);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x)
+                        ov[x] = fmaf(ec, __uint_as_float(re[8 * h + x]), gi * __uint_as_float(ri[8 * h + x]));
+                    if (store) {
+                        if (OUT_F32) {
+                            float4* dst = reinterpret_cast<float4*>(
+                                static_cast<float*>(p.o) + orow * D + 16 * c + 8 * h);
+                            dst[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
+                            dst[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
+                        } else {
+                            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow * D +
+                                                      16 * c + 8 * h) =
+                                make_uint4(pack_bf16x2(ov[0], ov[1]), pack_bf16x2(ov[2], ov[3]),
+                                           pack_bf16x2(ov[4], ov[5]), pack_bf16x2(ov[6], ov[7]));
+                        }
                     }
                 }
             }
@@ -1117,8 +1175,8 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
 
 // Small shared state at the start of the dynamic region; the 1024-aligned
 // tile region follows (SMEM_BYTES reserves the worst-case alignment gap).
-constexpr uint32_t SM_BARS = 0;                       // 32 x 8 B
-constexpr uint32_t SM_RING = 256;                     // 2 x Item
+constexpr uint32_t SM_BARS = 0;                       // 36 x 8 B
+constexpr uint32_t SM_RING = 288;                     // 2 x Item
 constexpr uint32_t SM_PW = 384;                       // (C+1) floats
 constexpr uint32_t SM_SC = 912;                       // 4 x ScaleRec (144 B)
 constexpr uint32_t SM_RED = SM_SC + 4 * 144;          // 16 floats
@@ -1126,7 +1184,7 @@ constexpr uint32_t SM_HS = SM_RED + 64;               // [2][128] bytes
 constexpr uint32_t SM_TMEM = SM_HS + 256;             // u32
 constexpr uint32_t SM_ABORT = SM_TMEM + 4;            // int
 constexpr uint32_t SM_SMALL = SM_ABORT + 4;
-static_assert(NUM_BARS <= 32, "barrier area");
+static_assert(NUM_BARS <= 36, "barrier area");
 static_assert(sizeof(Item) * 2 <= SM_PW - SM_RING, "ring area");
 static_assert(SM_PW + (C + 1) * 4 <= SM_SC, "pw area");
 static_assert(sizeof(ScaleRec) == 144, "scale record");
@@ -1161,7 +1219,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         counts[B_FULL0] = counts[B_FULL1] = counts[B_EMPTY0] = counts[B_EMPTY1] = 1;
         counts[B_SBLK_FULL] = counts[B_SB_FREE] = counts[B_O_FULL] = counts[B_DS_FULL] = 1;
         counts[B_ITEM_FULL0] = counts[B_ITEM_FULL1] = counts[B_FIN] = 1;
-        counts[B_ITEM_EMPTY0] = counts[B_ITEM_EMPTY1] = 13;  // MMA lane + 12 group warps
+        counts[B_QFULL0] = counts[B_QFULL1] = 1;
+        counts[B_ITEM_EMPTY0] = counts[B_ITEM_EMPTY1] = 15;  // MMA lane + 14 group warps
+        // Q converters (64 threads) join the K/V converters (128).
+        counts[B_CONV0] = counts[B_CONV1] = 192;
+        counts[B_SC_FULL0] = counts[B_SC_FULL1] = counts[B_SC_FULL2] = counts[B_SC_FULL3] = 192;
         for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], counts[i]);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tq)) : "memory");
@@ -1183,6 +1245,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_CTRL));
         if (warp == 0 && lane == 0) producer_role(p, &tq, &tk, &tv, sm);
         if (warp == 1 && lane == 0) mma_role(p, sm, tmem);
+        if (warp >= 2) qcv_role(p, sm, warp, lane);
     } else if (warp < 8) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_CV));
         cv_role(p, sm, warp, lane);

@@ -1,0 +1,118 @@
+"""Parity at the benchmark's full sizes, in the launch configuration bench.py
+times (default tuning), against the fp64 oracle on sampled heads and rows.
+
+Workloads (seeded, synthetic):
+  * MiniMax-shaped prefill: B=1, H=64, N=32768, d=128, bf16;
+  * varlen batched prefill: 16 sequences, lengths uniform in [1024, 65536];
+  * long-context prefill: N = 1,048,576;
+  * decode, batch 256, fp32 state [256,64,128,128], and the backward pass on the
+    MiniMax prefill shape.
+The oracle computes whole heads by its token recurrence (pinned against the
+quadratic form) and single rows by the quadratic form itself.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_02_b200 import binding as L
+from long_context_02_b200 import inputs
+from tests.gpu_util import (TOL_BF16, assert_close, assert_close_bf16_out, f64, lam)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+SAMPLE_HEADS = [0, 21, 42, 63]
+
+
+@pytest.fixture(autouse=True)
+def _default_tuning():
+    L.la_set_tuning(0, 0)
+    yield
+    torch.cuda.empty_cache()
+
+
+def _heads(t, hs):
+    return np.stack([f64(t[0, h]) for h in hs])[None]
+
+
+def test_minimax_prefill_32k():
+    B, H, N, d = 1, 64, 32768, 128
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.bfloat16, DEV, seed=1000)
+    o = torch.empty(q.shape, dtype=torch.float32, device=DEV)
+    ob = torch.empty_like(q)
+    st = torch.empty((B, H, d, d), dtype=torch.float32, device=DEV)
+    ws = L.workspace(L.LA_OP_PREFILL, B, H, N, d)
+    L.la_prefill(q, k, v, s, o, st, ws)
+    L.la_prefill(q, k, v, s, ob, None, ws)
+    assert L.la_read_device_status(ws) == L.LA_OK
+    hs = SAMPLE_HEADS
+    o_ref, st_ref = oracle.recurrence(_heads(q, hs), _heads(k, hs), _heads(v, hs), lam(s)[hs])
+    assert_close(_heads(o, hs), o_ref, TOL_BF16, "O (sampled heads)")
+    assert_close(np.stack([f64(st[0, h]) for h in hs])[None], st_ref, TOL_BF16, "state")
+    assert_close_bf16_out(_heads(ob, hs), o_ref, TOL_BF16, "bf16 O (sampled heads)")
+    # Single rows by the quadratic form (segment and block boundaries, the end).
+    rows = [0, 127, 128, 2047, 2048, 16383, 16384, N - 1]
+    for h in (0, 63):
+        want = oracle.forward_rows(f64(q[0, h]), f64(k[0, h]), f64(v[0, h]), lam(s)[h], rows)
+        got = f64(o[0, h])[rows]
+        rms = float(np.sqrt(np.mean(o_ref[0, hs.index(h)] ** 2)))
+        assert np.max(np.abs(got - want)) <= TOL_BF16 * rms, f"rows of head {h}"
+
+
+def test_varlen_16_sequences():
+    H, d = 64, 128
+    lengths = inputs.varlen_lengths(16, 1024, 65536, seed=0)
+    q, k, v, cu, s = inputs.varlen_inputs(lengths, H, d, torch.bfloat16, DEV, seed=1001)
+    T = q.shape[1]
+    o = torch.empty(q.shape, dtype=torch.float32, device=DEV)
+    st = torch.empty((16, H, d, d), dtype=torch.float32, device=DEV)
+    ws = L.workspace(L.LA_OP_PREFILL_VARLEN, 1, H, T, d, 16)
+    L.la_prefill_varlen(cu, q, k, v, s, o, st, ws)
+    assert L.la_read_device_status(ws) == L.LA_OK
+    hs = [0, 63]
+    sub = lambda t: np.stack([f64(t[h]) for h in hs])
+    o_ref, st_ref = oracle.recurrence_varlen(cu.cpu().numpy(), sub(q), sub(k), sub(v),
+                                             lam(s)[hs])
+    assert_close(sub(o), o_ref, TOL_BF16, "O (heads 0, 63)")
+    assert_close(np.stack([f64(st[:, h]) for h in hs], axis=1), st_ref, TOL_BF16, "states")
+
+
+def test_long_context_1m():
+    B, H, N, d = 1, 64, 1 << 20, 128
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.bfloat16, DEV, seed=1002)
+    o = torch.empty_like(q)
+    st = torch.empty((B, H, d, d), dtype=torch.float32, device=DEV)
+    ws = L.workspace(L.LA_OP_PREFILL, B, H, N, d)
+    L.la_prefill(q, k, v, s, o, st, ws)
+    assert L.la_read_device_status(ws) == L.LA_OK
+    # Head 63 has the slowest decay (the scan carries the most state) and
+    # head 0 the fastest; whole heads by the recurrence.
+    hs = [0, 63]
+    o_ref, st_ref = oracle.recurrence(_heads(q, hs), _heads(k, hs), _heads(v, hs), lam(s)[hs])
+    assert_close_bf16_out(_heads(o, hs), o_ref, TOL_BF16, "bf16 O (heads 0, 63)")
+    assert_close(np.stack([f64(st[0, h]) for h in hs])[None], st_ref, TOL_BF16, "state")
+
+
+def test_decode_batch_256():
+    B, H, d = 256, 64, 128
+    q, k, v, state, s = inputs.decode_inputs(B, H, d, torch.bfloat16, DEV, seed=1003)
+    st_in = f64(state)
+    o = torch.empty(q.shape, dtype=torch.float32, device=DEV)
+    L.la_decode(q, k, v, s, state, o)
+    o_ref, st_ref = oracle.decode(f64(q), f64(k), f64(v), lam(s), st_in)
+    assert_close(f64(o), o_ref, TOL_BF16, "o")
+    assert_close(f64(state), st_ref, TOL_BF16, "state")
+
+
+def test_backward_minimax_shape():
+    B, H, N, d = 1, 64, 32768, 128
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.bfloat16, DEV, seed=1004)
+    do = inputs.grad_output(q.shape, torch.bfloat16, DEV, seed=1005)
+    dq, dk, dv = L.backward(do, q, k, v, s, out_dtype=torch.float32)
+    hs = [0, 63]
+    rq, rk, rv = oracle.backward_recurrence(_heads(do, hs), _heads(q, hs), _heads(k, hs),
+                                            _heads(v, hs), lam(s)[hs])
+    assert_close(_heads(dq, hs), rq, TOL_BF16, "dQ")
+    assert_close(_heads(dk, hs), rk, TOL_BF16, "dK")
+    assert_close(_heads(dv, hs), rv, TOL_BF16, "dV")
