@@ -178,12 +178,21 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a per-rank scalar over all ranks (NCCL on GPUs, gloo on CPU)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank, local_ms, world):
+    """Aggregate throughput of `world` replicas: all units over the slowest rank's time.
+    Returns (max ms over ranks, units per second)."""
+    ms = max_over_ranks(local_ms, world)
+    return ms, world * units_per_rank / (ms * 1e-3)
 
 
 def timed(fn, steps, world, stream=None):
@@ -232,7 +241,7 @@ def run_ours(args):
 
     F = prefill_flops(B_, H_, N_)
     Bytes = prefill_bytes(B_, H_, N_)
-    value = world * F / (ms * 1e-3) / 1e12
+    value = world * F / (ms * 1e-3) / 1e12  # ms is already the max over ranks
     achieved = Bytes / (ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),

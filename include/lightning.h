@@ -158,6 +158,18 @@ LA_API int la_get_tuning(int* block_tokens, int* segment_tokens);
 LA_API int la_last_launch_count(void);
 
 /*
+ * Test-only fault injection for the chunk-parallel state scan of the bf16
+ * path, set on the host (process-wide, not thread-safe with concurrent calls).
+ *   skip_publish   non-zero: segments never signal that their prefix state is
+ *                  ready, so every later segment's bounded wait runs out
+ *   wait_limit_us  bound of that wait in microseconds (0 = default, 2 s)
+ * An expired wait is reported as LA_ERR_TIMEOUT by la_read_device_status;
+ * the outputs of that call are then invalid, the CUDA context stays usable.
+ * Call la_set_fault_injection(0, 0) to restore normal operation.
+ */
+LA_API int la_set_fault_injection(int skip_publish, int wait_limit_us);
+
+/*
  * Size in bytes of the scratch array built into the library for
  * la_prefill_noalloc (16 MiB).
  */

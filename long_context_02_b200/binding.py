@@ -25,7 +25,7 @@ LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE, LA_OP_BACKWARD = 0, 1, 2, 3
 
 EXPORTED = ["la_workspace_bytes", "la_prefill", "la_prefill_varlen", "la_decode", "la_backward",
             "la_status_string", "la_read_device_status", "la_set_tuning", "la_get_tuning",
-            "la_last_launch_count", "la_prefill_noalloc"]
+            "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection"]
 
 _lib = None
 
@@ -58,9 +58,10 @@ def lib():
         L.la_get_tuning.argtypes = [ctypes.POINTER(I), ctypes.POINTER(I)]
         L.la_last_launch_count.argtypes = []
         L.la_prefill_noalloc.argtypes = [P, P, P, P, P, P, I, I, LL, I, I, I, P]
+        L.la_set_fault_injection.argtypes = [I, I]
         for f in ("la_prefill", "la_prefill_varlen", "la_decode", "la_backward",
                   "la_read_device_status", "la_set_tuning", "la_get_tuning",
-                  "la_last_launch_count", "la_prefill_noalloc"):
+                  "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -153,6 +154,12 @@ def la_get_tuning():
     b, s = ctypes.c_int(), ctypes.c_int()
     lib().la_get_tuning(ctypes.byref(b), ctypes.byref(s))
     return b.value, s.value
+
+
+def la_set_fault_injection(skip_publish=0, wait_limit_us=0):
+    """Test-only: make the scan's inter-segment waits run out (see lightning.h)."""
+    _check("la_set_fault_injection", lib().la_set_fault_injection(int(skip_publish),
+                                                                 int(wait_limit_us)))
 
 
 def la_last_launch_count() -> int:

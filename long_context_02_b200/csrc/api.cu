@@ -251,4 +251,12 @@ LA_API int la_get_tuning(int* block_tokens, int* segment_tokens)
 
 LA_API int la_last_launch_count(void) { return g_launches; }
 
+LA_API int la_set_fault_injection(int skip_publish, int wait_limit_us)
+{
+    if (wait_limit_us < 0) return LA_ERR_INVALID_ARG;
+    g_fault.skip_publish = skip_publish ? 1 : 0;
+    g_fault.wait_limit_us = wait_limit_us;
+    return LA_OK;
+}
+
 }  // extern "C"

@@ -131,6 +131,8 @@ struct Params {
     WsHeader* hdr;
     int* chain_flags;   // per chain: segments published so far
     float* incl;        // [chains][2][D][D] inclusive prefixes (ring of two)
+    unsigned long long flag_limit_ns;  // bound of the inter-CTA wait
+    int skip_publish;   // fault injection (tests): never raise the chain counters
 };
 
 struct Item {
@@ -1070,7 +1072,7 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
                     if (seen >= it.p_ord) break;
                     if ((spin & 15) == 15) {
                         if (*sm.abort) break;
-                        if (globaltimer() - t0 > FLAG_LIMIT_NS) {
+                        if (globaltimer() - t0 > p.flag_limit_ns) {
                             atomicExch(&p.hdr->status, (int)LA_ERR_TIMEOUT);
                             break;
                         }
@@ -1103,7 +1105,7 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         if (has_succ) {
             __threadfence();
             if (!group_sync(&bars[B_OS_SYNC], n_sync, sm.abort, p.hdr)) break;
-            if (a == 0) {
+            if (a == 0 && !p.skip_publish) {
                 int* flag = p.chain_flags + it.chain;
                 asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(it.p_ord + 1) : "memory");
             }
@@ -1423,6 +1425,8 @@ static WsLayout layout(const Problems& P, int seg, bool varlen)
 
 }  // namespace tc
 
+FaultInjection g_fault;
+
 size_t tc_workspace_bytes(const Problems& P, int d, int seg_tuning, bool varlen)
 {
     (void)d;
@@ -1468,6 +1472,9 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     prm.hdr = reinterpret_cast<WsHeader*>(ws);
     prm.chain_flags = reinterpret_cast<int*>(ws + w.flags);
     prm.incl = reinterpret_cast<float*>(ws + w.incl);
+    prm.flag_limit_ns = g_fault.wait_limit_us > 0 ? 1000ull * (unsigned long long)g_fault.wait_limit_us
+                                                   : FLAG_LIMIT_NS;
+    prm.skip_publish = g_fault.skip_publish;
 
     CUtensorMap mq, mk, mv;
     const unsigned long long dim1 = varlen ? (unsigned long long)std::max<long long>(P.total, 1)

@@ -8,6 +8,13 @@
 
 namespace la {
 
+// Test-only fault injection (set through la_set_fault_injection).
+struct FaultInjection {
+    int skip_publish = 0;   // segments never publish their prefix: successors time out
+    int wait_limit_us = 0;  // bound of the inter-CTA wait (0 = default, 2 s)
+};
+extern FaultInjection g_fault;
+
 // Workspace bytes after the header: per-chain flags, two inclusive-prefix
 // state slots per chain, and (varlen) the planned work items.
 size_t tc_workspace_bytes(const Problems& P, int d, int seg_tuning, bool varlen);
