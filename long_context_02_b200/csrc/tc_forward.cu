@@ -1,57 +1,57 @@
 // Lightning attention on the sm_100a tensor cores: tcgen05 MMAs with TMEM
-// accumulators, TMA-staged tiles, a chunk-parallel scan of the d x d state
-// across segments, bf16 inputs, head dim 128.
+// accumulators, TMA-staged bf16 tiles, a chunk-parallel scan of the state
+// across segments, head dim 128.
 //
 // What is computed (per (sequence, head) "chain", decay lam = exp(-slope)):
 //   O_i = sum_{j<=i} lam^(i-j) (q_i . k_j) v_j,   final state sum_j lam^(N-1-j) k_j^T v_j.
 // "MiniMax-01: Scaling Foundation Models with Lightning Attention | Summary":
 //   section 2.2 - tiles: a masked intra-tile product plus the product with the
 //                 accumulated key-value state, which is then updated;
-//   section 3.2 - LASP+: each partition summarizes its keys/values locally, the
-//                 summaries are combined into global prefixes, so partitions
-//                 need not wait for the full serial pass before them;
-//   section 3.3 - tiles of 32..256 tokens, batched matmuls (here tcgen05).
+//   section 3.2 - LASP+: each partition summarizes its keys/values locally and
+//                 the summaries combine into prefixes, so partitions need not
+//                 wait for the serial pass before them;
+//   section 3.3 - tiled prefill on batched matmuls (here tcgen05).
 //
-// Work decomposition. A chain of N tokens is cut into segments of SEG tokens
-// (a multiple of the 128-token block). A work item is one (chain, segment).
-// Persistent CTAs (one per SM) take items from an atomic ticket in
-// segment-major order, so an item's predecessor in its chain always holds a
-// smaller ticket and is already running or done. For each item:
-//   phase A (if a later segment needs it): the segment's local state
-//     S_loc = sum_j lam^(len-1-j) k_j^T v_j, block by block; then wait for the
-//     predecessor's inclusive prefix S_prev (bounded spin on a per-chain
-//     counter) and publish S_incl = lam^len S_prev + S_loc: the scan combine
+// Work decomposition. The value dimension is split in two halves of 64
+// columns: O[:, half] and state[:, half] need only V[:, half], so each
+// (chain, half) is an independent problem with its own 128 x 64 state. A
+// chain is also cut into segments of SEG tokens (a multiple of the 128-token
+// block; one segment when there are enough chains to fill the GPU). A work
+// item is one (chain, half, segment). Persistent CTAs (one per SM) take items
+// from an atomic ticket in segment-major order, so an item's predecessor in
+// its chain always holds a smaller ticket and is already running or done.
+// For each item:
+//   phase A (only if a later segment needs it): the segment's local state
+//     S_loc = sum_j lam^(len-1-j) k_j^T v_j, accumulated in TMEM over the
+//     segment's blocks; then a bounded wait for the predecessor's inclusive
+//     prefix S_prev and a publish of lam^len S_prev + S_loc: the scan combine
 //     (a1, S1) o (a2, S2) = (a1 a2, a2 S1 + S2).
-//   phase C: run the segment's 128-token blocks from S_in = S_prev:
-//     MMA1  SB  = Q K^T                     (fp32 in TMEM)
-//     E_P   P   = SB * lam^(i-j) [j<=i]      (fp16, written back into TMEM)
-//     MMA2  OI  = P V                       (A operand from TMEM)
-//     MMA3  OE  = Q S                       (S: fp32 state kept in registers)
-//     E_O   O   = OI + lam^(i+1) OE          -> global (bf16 or fp32)
-//     E_K   Kt  = lam^(L-1-j) k_j            (in place in shared memory)
-//     MMA4  DS^T = V^T Kt
-//     E_S   S   = lam^L S + DS               (fp32, registers; fp16 copy for MMA3)
-// Only non-negative decay exponents <= the block length appear, so nothing
-// overflows; terms that underflow are below fp32 resolution of the result.
+//   phase C: the segment's blocks from S = S_prev. Per 128-token block:
+//     MMA1  SP  = Q K^T                    (fp32, TMEM)
+//     E_P   P   = SP * lam^(i-j) [j<=i]     written back into TMEM as bf16 hi + lo
+//     MMA2  OI  = P_hi V + P_lo V           (A operand from TMEM)
+//     MMA3  OE  = Q S_hi + Q S_lo           (bf16 hi + lo copies of the fp32 state)
+//     E_O   O   = OI + lam^(i+1) OE  -> global (bf16 or fp32)
+//     E_V   Vd  = lam^(L-1-j) v_j           (bf16 hi + lo, shared memory)
+//     MMA4  DS  = K^T Vd_hi + K^T Vd_lo
+//     E_S   S   = lam^L S + DS              (fp32 in registers; hi + lo copies for MMA3)
+// Only non-negative decay exponents appear, so nothing overflows; terms that
+// underflow are below fp32 resolution of the result.
 //
-// Precision. Every tensor-core operand is fp16 with exact power-of-two
-// scaling: the relative rounding of the operands the kernel forms itself (P,
-// the state copy, the decayed keys) is 2^-11 (bf16 would be 2^-8, too coarse
-// for a max error of 1e-2 of rms), and fp16's narrow exponent range never
-// bites. As tiles land, converter warps rewrite Q (one scale per row), K and
-// V (one scale per tile) as fp16 in [1, 2) magnitude; the bf16 -> fp16 step
-// is exact. Then Q K^T is bounded by 512, so P needs no rescaling, and the
-// decayed keys are bounded by the K tile. Each column of the state copy has
-// its own scale (the state is held transposed, one value column per thread,
-// so that is a thread-local choice). All scales are undone in fp32 in the
-// epilogues.
+// Precision. Q, K and V enter the MMAs exactly as given (bf16). Every operand
+// the kernel forms itself (P, the state copy, the decayed values) is split as
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi): a relative error of about
+// 2^-16, with fp32's exponent range, so no scaling is needed anywhere. One
+// bf16 rounding of any of those three operands would cost about 1e-2 of the
+// output's rms; the split costs a second MMA for each.
 //
-// Warp roles (16 warps, 4 warpgroups): warp 0 TMA producer, warp 1 MMA
-// issuer (also owns TMEM), warps 2-3 Q converters; 4-7 K/V converters (fp16
-// tiles as they land); 8-11 "PE" (E_P and E_K after Q K^T); 12-15 "OS" (E_O,
-// E_S and the scan). TMEM: 512 columns = SB/P | OI | OE | DS^T, 128 lanes.
-// Shared memory: 2 stages x (Q, K, V) 128x128 16-bit tiles + the fp16 state
-// copy, all in the 128-byte-swizzled layout TMA writes.
+// Warp roles (16 warps, 4 warpgroups): warp 0 TMA producer, warp 1 MMA issuer
+// (also owns TMEM); warps 4-7 "P" (E_P); warps 8-11 "VO" (E_V, E_O); warps
+// 12-15 "S" (E_S and the scan; the fp32 state lives in their registers, one
+// key row a per thread). TMEM: 512 columns = SP[2] | OI | DS | OE[2].
+// Shared memory: two slots each for Q, K (128 x 128) and V (128 x 64), the
+// decayed values (hi, lo) and the state copies (hi, lo), all in the 128-byte
+// swizzled layout TMA writes.
 //
 // Every wait is bounded: an mbarrier wait gives up after 4 s, the inter-CTA
 // wait after 2 s; either records LA_ERR_TIMEOUT in the workspace header and
@@ -69,50 +69,61 @@ namespace la {
 namespace tc {
 
 constexpr int D = 128;                           // head dim (d_k = d_v)
+constexpr int DV = 64;                           // value columns per work item
 constexpr int C = 128;                           // tokens per block
 constexpr int NUM_THREADS = 512;                 // 4 warpgroups
 // Register split (setmaxnreg, which ptxas also uses to allocate each role):
-// launched at 65536 / 512 = 128 per thread, i.e. 65536 per CTA. The control
-// warpgroup drops to 64, the converters to 104, the PE group to 112, the OS
-// group rises to 232: 128 * (64 + 104 + 112 + 232) = 65536, and per SM
-// sub-partition (one warp of each group) 32 * 512 = 16384.
-constexpr int REGS_CTRL = 64, REGS_CV = 104, REGS_PE = 112, REGS_OS = 232;
+// launched at 65536 / 512 = 128 per thread. 128 * (96 + 120 + 120 + 168) =
+// 64512 <= 65536.
+constexpr int REGS_CTRL = 96, REGS_P = 120, REGS_VO = 120, REGS_S = 168;
 constexpr uint32_t BOX_BYTES = 128 * 64 * 2;     // one TMA box: 128 rows x 64 bf16
 constexpr uint32_t TILE_BYTES = 2 * BOX_BYTES;   // 128 x 128 bf16
-constexpr uint32_t STAGE_BYTES = 3 * TILE_BYTES; // Q, K, V
-constexpr uint32_t SMEM_TILES = 2 * STAGE_BYTES + TILE_BYTES;
+// Tile region (1024-aligned).
+constexpr uint32_t OFF_Q = 0;                          // 2 x 32 KB
+constexpr uint32_t OFF_K = OFF_Q + 2 * TILE_BYTES;     // 2 x 32 KB
+constexpr uint32_t OFF_V = OFF_K + 2 * TILE_BYTES;     // 2 x 16 KB
+constexpr uint32_t OFF_VH = OFF_V + 2 * BOX_BYTES;     // decayed values, hi
+constexpr uint32_t OFF_VL = OFF_VH + BOX_BYTES;        // decayed values, lo
+constexpr uint32_t OFF_SH = OFF_VL + BOX_BYTES;        // state copy, hi
+constexpr uint32_t OFF_SL = OFF_SH + BOX_BYTES;        // state copy, lo
+constexpr uint32_t SMEM_TILES = OFF_SL + BOX_BYTES;    // 224 KB
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_SB = 0, COL_OI = 128, COL_OE = 256, COL_DS = 384;
+constexpr uint32_t COL_SP = 0, COL_OI = 256, COL_DS = 320, COL_OE = 384;
 constexpr unsigned long long WAIT_LIMIT_NS = 4000000000ull;
 constexpr unsigned long long FLAG_LIMIT_NS = 2000000000ull;
 constexpr unsigned long long DRAIN_LIMIT_NS = 200000000ull;
 
+// Barriers. A waiter must never fall two phases behind its barrier (a parity
+// wait would then return at once or hang), so every resource that can be
+// two uses ahead of its consumer has one barrier per buffer.
 enum {
-    B_FULL0, B_FULL1, B_EMPTY0, B_EMPTY1, B_CONV0, B_CONV1, B_KT0, B_KT1, B_SBLK_FULL,
-    B_SB_FREE, B_P_READY, B_O_FULL, B_O_EMPTY, B_DS_FULL, B_DS_EMPTY, B_S_READY, B_SC_FULL0,
-    B_SC_FULL1, B_SC_FULL2, B_SC_FULL3, B_SC_EMPTY0, B_SC_EMPTY1, B_SC_EMPTY2, B_SC_EMPTY3,
-    B_ITEM_FULL0, B_ITEM_FULL1, B_ITEM_EMPTY0, B_ITEM_EMPTY1, B_FIN, B_CV_SYNC, B_PE_SYNC,
-    B_OS_SYNC, B_QFULL0, B_QFULL1, NUM_BARS
+    B_QF0, B_QF1, B_QE0, B_QE1,      // Q slots: loaded / released (after MMA3)
+    B_KF0, B_KF1, B_KE0, B_KE1,      // K slots: loaded / released (after MMA4)
+    B_VF0, B_VF1, B_VE0, B_VE1,      // V slots: loaded / released (after MMA2)
+    B_SP_FULL0, B_SP_FULL1,          // MMA1 done -> E_P
+    B_P_READY0, B_P_READY1,          // E_P done -> MMA2
+    B_VH_FREE, B_VH_READY,           // decayed values: MMA4 done / E_V done
+    B_DS_FULL, B_DS_EMPTY,           // DS: MMA4 done / E_S read it
+    B_S_FREE, B_S_READY,             // state copy: MMA3 done / E_S wrote it
+    B_O_FULL, B_O_EMPTY,             // OI, OE: MMA2 done / E_O read them
+    B_ITEM_FULL0, B_ITEM_FULL1, B_ITEM_EMPTY0, B_ITEM_EMPTY1,
+    B_FIN, B_P_SYNC, B_S_SYNC,
+    NUM_BARS
 };
-// A barrier's waiter must not skip phases: a parity wait on a barrier two
-// phases behind returns at once. So the Q tile, which only phase-C blocks
-// load, completes its own B_QFULL barrier rather than B_FULL, which every
-// block completes and the Q converters would otherwise skip in phase A.
 
-// tcgen05 instruction descriptors (kind::f16): D fp32, M = N = 128.
+// tcgen05 instruction descriptors (kind::f16): D fp32, M = 128, A and B bf16.
 // bits: [4,6) D format (1 = f32), [7,10) A format and [10,13) B format
-// (0 = f16, 1 = bf16; A and B always share one type), 15 A major, 16 B major
-// (0 = K-major, 1 = MN-major), [17,23) N >> 3, [24,29) M >> 4.
-constexpr uint32_t idesc(uint32_t fmt, uint32_t a_mn_major, uint32_t b_mn_major)
+// (1 = bf16), 15 A major, 16 B major (0 = K-major, 1 = MN-major),
+// [17,23) N >> 3, [24,29) M >> 4.
+constexpr uint32_t idesc(uint32_t n, uint32_t a_mn_major, uint32_t b_mn_major)
 {
-    return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
-           ((128u >> 3) << 17) | ((128u >> 4) << 24);
+    return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
+           ((n >> 3) << 17) | ((128u >> 4) << 24);
 }
-constexpr uint32_t F16 = 0, BF16 = 1;
-constexpr uint32_t IDESC_QK = idesc(F16, 0, 0);   // Q K^T: both K-major
-constexpr uint32_t IDESC_PV = idesc(F16, 0, 1);   // P (TMEM) V: V MN-major
-constexpr uint32_t IDESC_QS = idesc(F16, 0, 0);   // Q S: S stored as rows of S^T (K-major)
-constexpr uint32_t IDESC_VK = idesc(F16, 1, 1);   // V^T Kt: both MN-major
+constexpr uint32_t IDESC_QK = idesc(128, 0, 0);  // Q K^T: both K-major
+constexpr uint32_t IDESC_PV = idesc(64, 0, 1);   // P (TMEM) V: V MN-major
+constexpr uint32_t IDESC_QS = idesc(64, 0, 1);   // Q S: S rows = key dim, MN-major
+constexpr uint32_t IDESC_KV = idesc(64, 1, 1);   // K^T Vd: both MN-major
 
 struct Params {
     int H;
@@ -122,15 +133,15 @@ struct Params {
     long long N;        // dense: tokens per chain
     const int* cu_seqlens;  // varlen when not null
     long long total;
-    const int4* items;  // varlen: planned items {chain, p_ord, nseg, 0}
+    const int4* items;  // varlen: planned (chain, p_ord, nseg) per (chain, segment)
     int num_items_dense;
     const float* slopes;
     void* o;
     float* state_out;
     int reverse;
     WsHeader* hdr;
-    int* chain_flags;   // per chain: segments published so far
-    float* incl;        // [chains][2][D][D] inclusive prefixes (ring of two)
+    int* chain_flags;   // per (chain, half): segments published so far
+    float* incl;        // [chains][2 halves][2 slots][D][DV] inclusive prefixes
     unsigned long long flag_limit_ns;  // bound of the inter-CTA wait
     int skip_publish;   // fault injection (tests): never raise the chain counters
 };
@@ -138,6 +149,7 @@ struct Params {
 struct Item {
     int valid;
     int chain;
+    int half;           // value columns [64 half, 64 half + 64)
     int head;
     int p_ord;          // position in the chain's processing order
     int nseg;
@@ -195,8 +207,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity)
 // after `limit` ns, in which case it records the timeout and raises the
 // CTA-wide abort flag.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort,
-                                       WsHeader* hdr,
-                                       unsigned long long limit = WAIT_LIMIT_NS)
+                                          WsHeader* hdr,
+                                          unsigned long long limit = WAIT_LIMIT_NS)
 {
     if (mbar_try_wait(b, parity)) return true;
     const unsigned long long t0 = globaltimer();
@@ -213,13 +225,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
     }
 }
 
-__device__ __forceinline__ void fence_proxy_async()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Warp-uniform bounded wait for the 4-warp epilogue groups: every lane polls,
-// and the warp proceeds only if all lanes saw the phase complete.
+// Warp-uniform bounded wait: every lane polls, and the warp proceeds only if
+// all lanes saw the phase complete.
 __device__ __forceinline__ bool wait_warp(uint64_t* b, uint32_t parity, volatile int* abort,
                                           WsHeader* hdr)
 {
@@ -227,7 +234,7 @@ __device__ __forceinline__ bool wait_warp(uint64_t* b, uint32_t parity, volatile
     return __all_sync(0xffffffffu, ok);
 }
 
-// Bounded barrier over one 128-thread epilogue group (an mbarrier of count 128).
+// Bounded barrier over one 128-thread group (an mbarrier of count 128).
 __device__ __forceinline__ bool group_sync(uint64_t* b, uint32_t& n, volatile int* abort,
                                            WsHeader* hdr)
 {
@@ -235,13 +242,38 @@ __device__ __forceinline__ bool group_sync(uint64_t* b, uint32_t& n, volatile in
     return wait_warp(b, n++ & 1, abort, hdr);
 }
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                            int y, int z)
+__device__ __forceinline__ void fence_proxy_async()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_normal()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y, int z, uint64_t policy)
 {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)),
+        "l"(policy)
         : "memory");
 }
 
@@ -296,27 +328,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-        "%11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
-{
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                   "=r"(r[6]), "=r"(r[7])
-                 : "r"(taddr)
-                 : "memory");
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
 {
     asm volatile(
@@ -342,6 +353,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 __device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
+// x0, x1 -> (hi, lo) bf16x2 words with x = hi + lo to about 2^-16 relative.
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo)
+{
+    hi = pack_bf16x2(x0, x1);
+    lo = pack_bf16x2(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
+}
+
 // Shared-memory matrix descriptor: 128-byte swizzle, sm_100 version bit.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
 {
@@ -349,17 +367,25 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// K-major 128x128 tile (two 64-column boxes): k-step ks covers K elements [16ks, 16ks+16).
+// K-major 128 x 128 tile (two 64-column boxes): k-step ks covers K elements [16ks, 16ks+16).
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int ks)
 {
     return sdesc(tile + (uint32_t)(ks >> 2) * BOX_BYTES + (uint32_t)(ks & 3) * 32u, 16u, 1024u);
 }
 
-// MN-major 128x128 tile (rows = K dim, two 64-element boxes along MN):
-// k-step ks covers rows [16ks, 16ks+16).
+// MN-major tile with rows = K dim and two 64-element boxes along MN,
+// BOX_BYTES apart (the leading byte offset): k-step ks covers rows
+// [16ks, 16ks+16).
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int ks)
 {
     return sdesc(tile + (uint32_t)ks * 2048u, BOX_BYTES, 1024u);
+}
+
+// MN-major box, 64 elements wide (one swizzle atom along MN, so the leading
+// byte offset is not used; it is kept small and in bounds).
+__device__ __forceinline__ uint64_t desc_mn64(uint32_t box, int ks)
+{
+    return sdesc(box + (uint32_t)ks * 2048u, 16u, 1024u);
 }
 
 __device__ __forceinline__ int num_blocks(int len) { return (len + C - 1) / C; }
@@ -371,15 +397,13 @@ __device__ __forceinline__ int block_t0(int len, int k, int rev)
     return (rev ? nb - 1 - k : k) * C;
 }
 
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+// Offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled box.
+__device__ __forceinline__ uint32_t swz(int r, int c)
 {
-    uint32_t r;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
+    return (uint32_t)r * 128u + ((uint32_t)((c ^ r) & 7) << 4);
 }
 
-// Ordered L2 loads/stores (volatile asm keeps their program order, which
-// bounds how many values are in flight and stops loads being hoisted).
+// Ordered L2 loads/stores (volatile asm keeps their program order).
 __device__ __forceinline__ float4 ld_cg_ordered(const float* p)
 {
     float4 w;
@@ -396,86 +420,38 @@ __device__ __forceinline__ void st_cg_ordered(float* p, float4 w)
                  : "memory");
 }
 
-// Exact power-of-two scales for a max magnitude m: down * m lies in [1, 2),
-// up = 1 / down. Zero, subnormal or non-finite m keep scale 1.
-// `ue` is the biased fp32 exponent of `up` (how the scale is kept in shared memory).
-struct Pow2 {
-    float down, up;
-    uint8_t ue;
-};
-__device__ __forceinline__ Pow2 pow2_for(float m)
-{
-    const uint32_t e = (__float_as_uint(m) >> 23) & 0xffu;
-    if (e == 0u || e == 255u) return {1.f, 1.f, (uint8_t)127};
-    return {__uint_as_float((254u - e) << 23), __uint_as_float(e << 23), (uint8_t)e};
-}
-__device__ __forceinline__ float up_of(uint8_t ue) { return __uint_as_float((uint32_t)ue << 23); }
-
-// Offset of 16-byte chunk c (0..15) of row r in a 128x128 16-bit tile stored as
-// two 128-byte-swizzled 64-column boxes (the layout TMA writes).
-__device__ __forceinline__ uint32_t chunk_off(int r, int c)
-{
-    return (uint32_t)(c >> 3) * BOX_BYTES + (uint32_t)r * 128u + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
-}
-
-// Load row r of a bf16 tile as 128 floats.
-__device__ __forceinline__ void load_row_bf16(const uint8_t* tile, int r, float (&x)[128])
+// Write 64 fp32 values as hi and lo bf16 rows r of two swizzled 128 x 64 boxes.
+__device__ __forceinline__ void store_split_row(uint8_t* hi_box, uint8_t* lo_box, int r,
+                                                const float (&x)[DV])
 {
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        const uint4 w = *reinterpret_cast<const uint4*>(tile + chunk_off(r, c));
-        x[8 * c + 0] = bf16_lo(w.x); x[8 * c + 1] = bf16_hi(w.x);
-        x[8 * c + 2] = bf16_lo(w.y); x[8 * c + 3] = bf16_hi(w.y);
-        x[8 * c + 4] = bf16_lo(w.z); x[8 * c + 5] = bf16_hi(w.z);
-        x[8 * c + 6] = bf16_lo(w.w); x[8 * c + 7] = bf16_hi(w.w);
+    for (int c = 0; c < 8; ++c) {
+        uint4 h, l;
+        split2(x[8 * c + 0], x[8 * c + 1], h.x, l.x);
+        split2(x[8 * c + 2], x[8 * c + 3], h.y, l.y);
+        split2(x[8 * c + 4], x[8 * c + 5], h.z, l.z);
+        split2(x[8 * c + 6], x[8 * c + 7], h.w, l.w);
+        *reinterpret_cast<uint4*>(hi_box + swz(r, c)) = h;
+        *reinterpret_cast<uint4*>(lo_box + swz(r, c)) = l;
     }
-}
-
-// Store 128 floats times f as fp16 into row r of a tile.
-__device__ __forceinline__ void store_row_f16(uint8_t* tile, int r, const float (&x)[128], float f)
-{
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        uint4 w;
-        w.x = pack_f16x2(x[8 * c + 0] * f, x[8 * c + 1] * f);
-        w.y = pack_f16x2(x[8 * c + 2] * f, x[8 * c + 3] * f);
-        w.z = pack_f16x2(x[8 * c + 4] * f, x[8 * c + 5] * f);
-        w.w = pack_f16x2(x[8 * c + 6] * f, x[8 * c + 7] * f);
-        *reinterpret_cast<uint4*>(tile + chunk_off(r, c)) = w;
-    }
-}
-
-__device__ __forceinline__ float row_absmax(const float (&x)[128])
-{
-    float m = 0.f;
-#pragma unroll
-    for (int i = 0; i < 128; ++i) m = fmaxf(m, fabsf(x[i]));
-    return m;
-}
-
-// Convert row r of a bf16 tile in place to fp16 scaled to [1, 2); rows at or
-// beyond `valid` become zero. Returns the scale (`up` undoes it).
-__device__ __forceinline__ Pow2 convert_row(uint8_t* tile, int r, int valid)
-{
-    float x[128];
-    load_row_bf16(tile, r, x);
-    const Pow2 s = pow2_for(row_absmax(x));
-    store_row_f16(tile, r, x, r < valid ? s.down : 0.f);
-    return s;
 }
 
 // ------------------------------------------------------------------ work items
 
+// Ticket t -> (chain, half, segment). Halves of one (chain, segment) take
+// adjacent tickets, so they run side by side and share Q and K in L2.
 __device__ Item make_item(const Params& p, int t, int num_items)
 {
     Item it{};
     it.valid = 0;
     if (t >= num_items) return it;
+    const int base = t >> 1;
+    it.half = t & 1;
     int chain, p_ord, nseg;
     long long seq_start, seq_len, rowbase;
     if (p.cu_seqlens == nullptr) {
-        p_ord = t / p.nchains;
-        chain = t % p.nchains;
+        p_ord = base / p.nchains;
+        chain = base % p.nchains;
         nseg = p.nseg;
         it.head = chain % p.H;
         it.z = chain;
@@ -483,7 +459,7 @@ __device__ Item make_item(const Params& p, int t, int num_items)
         seq_len = p.N;
         rowbase = (long long)chain * p.N;
     } else {
-        const int4 w = p.items[t];
+        const int4 w = p.items[base];
         chain = w.x;
         p_ord = w.y;
         nseg = w.z;
@@ -508,67 +484,49 @@ __device__ Item make_item(const Params& p, int t, int num_items)
 
 // ------------------------------------------------------------------ roles
 
-// Scales of one loaded block, handed from the converter group to the OS group
-// through a ring of four slots (B_SC_FULL / B_SC_EMPTY). Each byte is the
-// biased fp32 exponent of the factor that undoes a power-of-two scaling.
-struct ScaleRec {
-    uint8_t qe[C];  // Q rows (phase-C blocks)
-    uint8_t kc;     // K tile (phase C: K as fed to Q K^T; phase A: decayed keys)
-    uint8_t vc;     // V tile
-    uint8_t pad[14];
-};
-
 struct Smem {
-    uint8_t* tiles;  // 1024-aligned: stage0 {Q,K,V}, stage1 {Q,K,V}, S16
+    uint8_t* tiles;  // 1024-aligned tile region
     uint64_t* bars;
     Item* ring;
     volatile int* abort;
-    float* pw_pe;    // [C+1] lam^m of the PE group's current item
-    ScaleRec* sc;    // [4]
-    float* red;      // [2][8] partial tile maxima of the converter group
-    uint8_t* hs;     // [2][4] state-copy scales, one per 32 columns (OS group)
-    __device__ uint8_t* q(int s) const { return tiles + s * STAGE_BYTES; }
-    __device__ uint8_t* k(int s) const { return tiles + s * STAGE_BYTES + TILE_BYTES; }
-    __device__ uint8_t* v(int s) const { return tiles + s * STAGE_BYTES + 2 * TILE_BYTES; }
-    __device__ uint8_t* s16() const { return tiles + 2 * STAGE_BYTES; }
+    float* pw;       // [C+1] lam^m of the P group's current item
+    __device__ uint8_t* q(int s) const { return tiles + OFF_Q + s * TILE_BYTES; }
+    __device__ uint8_t* k(int s) const { return tiles + OFF_K + s * TILE_BYTES; }
+    __device__ uint8_t* v(int s) const { return tiles + OFF_V + s * BOX_BYTES; }
+    __device__ uint8_t* vh() const { return tiles + OFF_VH; }
+    __device__ uint8_t* vl() const { return tiles + OFF_VL; }
+    __device__ uint8_t* sh() const { return tiles + OFF_SH; }
+    __device__ uint8_t* sl() const { return tiles + OFF_SL; }
 };
 
-__device__ __forceinline__ uint64_t l2_policy_evict_first()
+// Reads the next item from the ring (all roles see the same sequence).
+__device__ __forceinline__ bool next_item(const Params& p, const Smem& sm, uint32_t k, Item& it,
+                                          bool warp_wide, int lane)
 {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-__device__ __forceinline__ uint64_t l2_policy_evict_last()
-{
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                                 int x, int y, int z, uint64_t policy)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)),
-        "l"(policy)
-        : "memory");
+    const int slot = k & 1;
+    const bool ok = warp_wide ? wait_warp(&sm.bars[B_ITEM_FULL0 + slot], (k >> 1) & 1, sm.abort, p.hdr)
+                              : mbar_wait(&sm.bars[B_ITEM_FULL0 + slot], (k >> 1) & 1, sm.abort, p.hdr);
+    if (!ok) return false;
+    it = sm.ring[slot];
+    if (warp_wide) __syncwarp();
+    if (!warp_wide || lane == 0) mbar_arrive(&sm.bars[B_ITEM_EMPTY0 + slot]);
+    return it.valid != 0;
 }
 
 __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUtensorMap* tk,
                               const CUtensorMap* tv, const Smem& sm)
 {
     uint64_t* bars = sm.bars;
-    const int num_items =
-        p.cu_seqlens ? *reinterpret_cast<volatile int*>(&p.hdr->num_items) : p.num_items_dense;
-    // K and V read in phase A are read again in phase C: keep them in L2;
-    // everything read for the last time goes first.
-    const uint64_t keep = l2_policy_evict_last(), drop = l2_policy_evict_first();
-    uint32_t n_load = 0;
-    uint32_t uses[2] = {0, 0}, quses[2] = {0, 0};
-    for (uint32_t k = 0;; ++k) {
+    const int num_items = 2 * (p.cu_seqlens ? *reinterpret_cast<volatile int*>(&p.hdr->num_items)
+                                            : p.num_items_dense);
+    // K and V read in phase A are read again in phase C: keep them in L2. Q
+    // and K are read by both halves of a chain; V only by its own half.
+    const uint64_t keep = l2_policy_evict_last(), normal = l2_policy_evict_normal(),
+                   drop = l2_policy_evict_first();
+    // nk, nv, nq: K, V and Q loads issued (K and V always come in pairs).
+    uint32_t nq = 0, nk = 0, nv = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
         const int slot = k & 1;
         if (!mbar_wait(&bars[B_ITEM_EMPTY0 + slot], ((k >> 1) & 1) ^ 1, sm.abort, p.hdr)) break;
         const int t = atomicAdd(&p.hdr->ticket, 1);
@@ -578,126 +536,167 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
         if (!it.valid) break;
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
-        bool ok = true;
         for (int pass = has_succ ? 0 : 1; pass < 2 && ok; ++pass) {
-            for (int kb = 0; kb < nb; ++kb) {
-                const int s = n_load & 1;
-                ok = mbar_wait(&bars[B_EMPTY0 + s], ((n_load >> 1) & 1) ^ 1, sm.abort, p.hdr);
-                if (!ok) break;
-                uint64_t* full = &bars[B_FULL0 + s];
+            const uint64_t kpol = pass ? normal : keep, vpol = pass ? drop : keep;
+            for (int kb = 0; kb < nb && ok; ++kb) {
                 const int y = it.y0 + block_t0(it.len, kb, p.reverse);
-                const uint64_t kv_pol = pass == 0 ? keep : drop;
-                mbar_expect_tx(full, 2 * TILE_BYTES);
+                const int s = nk & 1;
+                ok = mbar_wait(&bars[B_KE0 + s], ((nk >> 1) & 1) ^ 1, sm.abort, p.hdr);
+                if (!ok) break;
+                mbar_expect_tx(&bars[B_KF0 + s], TILE_BYTES);
+                tma_load_3d(sm.k(s), tk, &bars[B_KF0 + s], 0, y, it.z, kpol);
+                tma_load_3d(sm.k(s) + BOX_BYTES, tk, &bars[B_KF0 + s], 64, y, it.z, kpol);
+                ++nk;
                 if (pass == 1) {
-                    uint64_t* qfull = &bars[B_QFULL0 + s];
-                    mbar_expect_tx(qfull, TILE_BYTES);
-                    tma_load_3d_hint(sm.q(s), tq, qfull, 0, y, it.z, drop);
-                    tma_load_3d_hint(sm.q(s) + BOX_BYTES, tq, qfull, 64, y, it.z, drop);
-                    ++quses[s];
+                    const int sq = nq & 1;
+                    ok = mbar_wait(&bars[B_QE0 + sq], ((nq >> 1) & 1) ^ 1, sm.abort, p.hdr);
+                    if (!ok) break;
+                    mbar_expect_tx(&bars[B_QF0 + sq], TILE_BYTES);
+                    tma_load_3d(sm.q(sq), tq, &bars[B_QF0 + sq], 0, y, it.z, normal);
+                    tma_load_3d(sm.q(sq) + BOX_BYTES, tq, &bars[B_QF0 + sq], 64, y, it.z, normal);
+                    ++nq;
                 }
-                tma_load_3d_hint(sm.k(s), tk, full, 0, y, it.z, kv_pol);
-                tma_load_3d_hint(sm.k(s) + BOX_BYTES, tk, full, 64, y, it.z, kv_pol);
-                tma_load_3d_hint(sm.v(s), tv, full, 0, y, it.z, kv_pol);
-                tma_load_3d_hint(sm.v(s) + BOX_BYTES, tv, full, 64, y, it.z, kv_pol);
-                ++uses[s];
-                ++n_load;
+                ok = mbar_wait(&bars[B_VE0 + s], ((nv >> 1) & 1) ^ 1, sm.abort, p.hdr);
+                if (!ok) break;
+                mbar_expect_tx(&bars[B_VF0 + s], BOX_BYTES);
+                tma_load_3d(sm.v(s), tv, &bars[B_VF0 + s], DV * it.half, y, it.z, vpol);
+                ++nv;
             }
         }
-        if (!ok) break;
     }
     if (*sm.abort) {
-        // Wind down: let this CTA's copies in flight land before it exits.
-        for (int s = 0; s < 2; ++s)
-            if (uses[s] > 0) {
-                volatile int never = 0;
-                mbar_wait(&bars[B_FULL0 + s], (uses[s] - 1) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
-                if (quses[s] > 0)
-                    mbar_wait(&bars[B_QFULL0 + s], (quses[s] - 1) & 1, &never, p.hdr,
-                              DRAIN_LIMIT_NS);
-            }
+        // Wind down: let this CTA's copies in flight land before it exits
+        // (the last use of each slot; earlier uses completed before it).
+        volatile int never = 0;
+        for (uint32_t u = (nk > 2 ? nk - 2 : 0); u < nk; ++u)
+            mbar_wait(&bars[B_KF0 + (u & 1)], (u >> 1) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
+        for (uint32_t u = (nv > 2 ? nv - 2 : 0); u < nv; ++u)
+            mbar_wait(&bars[B_VF0 + (u & 1)], (u >> 1) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
+        for (uint32_t u = (nq > 2 ? nq - 2 : 0); u < nq; ++u)
+            mbar_wait(&bars[B_QF0 + (u & 1)], (u >> 1) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
     }
 }
 
 __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
 {
     uint64_t* bars = sm.bars;
-    const uint32_t s16 = smem_u32(sm.s16());
-    uint32_t n_load = 0, n_conv[2] = {0, 0}, n_kt[2] = {0, 0}, n_p = 0, n_c1 = 0, n_o = 0;
-    uint32_t n_s = 0, n_ds = 0;
-    // DS^T = V^T Kt for the block in stage s (fresh accumulator), then release the stage.
-    auto issue_vk = [&](int s) -> bool {
-        if (!mbar_wait(&bars[B_KT0 + s], n_kt[s]++ & 1, sm.abort, p.hdr)) return false;
-        if (!mbar_wait(&bars[B_DS_EMPTY], (n_ds++ & 1) ^ 1, sm.abort, p.hdr)) return false;
+    const uint32_t vh = smem_u32(sm.vh()), vl = smem_u32(sm.vl());
+    const uint32_t shi = smem_u32(sm.sh()), slo = smem_u32(sm.sl());
+    // nq, nkv: Q / K-V loads consumed; g: phase-C blocks; n_ds: DS productions;
+    // n_vh: decayed-value tiles; n_s: state copies.
+    uint32_t nq = 0, nkv = 0, g = 0, n_ds = 0, n_vh = 0, n_s = 0;
+    // DS = K^T Vd (hi and lo) for the K tile in slot sk.
+    auto mma4 = [&](int sk, bool accumulate) {
+        const uint32_t kk = smem_u32(sm.k(sk));
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ss(tmem + COL_DS, desc_mnmajor(kk, ks), desc_mn64(part ? vl : vh, ks),
+                       IDESC_KV, (accumulate || part || ks) ? 1u : 0u);
+    };
+    // SP[g & 1] = Q K^T for phase-C block g (Q slot nq, K slot nkv).
+    auto mma1 = [&](uint32_t gg, uint32_t q_use, uint32_t kv_use) -> bool {
+        const int sq = q_use & 1, sk = kv_use & 1;
+        if (!mbar_wait(&bars[B_QF0 + sq], (q_use >> 1) & 1, sm.abort, p.hdr)) return false;
+        if (!mbar_wait(&bars[B_KF0 + sk], (kv_use >> 1) & 1, sm.abort, p.hdr)) return false;
         tc_fence_after();
-        const uint32_t kk = smem_u32(sm.k(s)), vv = smem_u32(sm.v(s));
+        const uint32_t qq = smem_u32(sm.q(sq)), kk = smem_u32(sm.k(sk));
+        const uint32_t d = tmem + COL_SP + 128u * (gg & 1);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + COL_DS, desc_mnmajor(vv, ks), desc_mnmajor(kk, ks), IDESC_VK,
-                   ks > 0 ? 1u : 0u);
-        mma_commit(&bars[B_DS_FULL]);
-        mma_commit(&bars[B_EMPTY0 + s]);
+            mma_ss(d, desc_kmajor(qq, ks), desc_kmajor(kk, ks), IDESC_QK, ks > 0 ? 1u : 0u);
+        mma_commit(&bars[B_SP_FULL0 + (gg & 1)]);
         return true;
     };
-    // SB = Q K^T for the block in stage (nl & 1), once the converters are done with it.
-    auto issue_qk = [&](uint32_t nl) -> bool {
-        const int s = nl & 1;
-        if (!mbar_wait(&bars[B_CONV0 + s], n_conv[s]++ & 1, sm.abort, p.hdr)) return false;
-        if (!mbar_wait(&bars[B_SB_FREE], (n_c1++ & 1) ^ 1, sm.abort, p.hdr)) return false;
-        tc_fence_after();
-        const uint32_t qq = smem_u32(sm.q(s)), kk = smem_u32(sm.k(s));
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-            mma_ss(tmem + COL_SB, desc_kmajor(qq, ks), desc_kmajor(kk, ks), IDESC_QK,
-                   ks > 0 ? 1u : 0u);
-        mma_commit(&bars[B_SBLK_FULL]);
-        return true;
-    };
+    Item it;
     for (uint32_t k = 0;; ++k) {
-        const int slot = k & 1;
-        if (!mbar_wait(&bars[B_ITEM_FULL0 + slot], (k >> 1) & 1, sm.abort, p.hdr)) break;
-        const Item it = sm.ring[slot];
-        mbar_arrive(&bars[B_ITEM_EMPTY0 + slot]);
-        if (!it.valid) break;
+        if (!next_item(p, sm, k, it, false, 0)) break;
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
         if (has_succ) {
-            // Phase A: the segment's local state, block by block (accumulated by OS).
-            for (int b = 0; b < nb && ok; ++b) {
-                ok = issue_vk(n_load & 1);
-                ++n_load;
+            // Phase A: DS accumulates the segment's local state over its blocks.
+            for (int kb = 0; kb < nb && ok; ++kb) {
+                const int sk = nkv & 1;
+                ok = mbar_wait(&bars[B_KF0 + sk], (nkv >> 1) & 1, sm.abort, p.hdr) &&
+                     mbar_wait(&bars[B_VH_READY], n_vh & 1, sm.abort, p.hdr) &&
+                     (kb > 0 || mbar_wait(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr));
+                if (!ok) break;
+                ++n_vh;
+                tc_fence_after();
+                mma4(sk, kb > 0);
+                mma_commit(&bars[B_VH_FREE]);
+                mma_commit(&bars[B_KE0 + sk]);
+                mma_commit(&bars[B_VE0 + sk]);
+                ++nkv;
             }
             if (!ok) break;
+            mma_commit(&bars[B_DS_FULL]);
+            ++n_ds;
         }
         // Phase C.
-        if (!issue_qk(n_load)) break;
+        const uint32_t q0 = nq, kv0 = nkv, g0 = g;
+        if (!mma1(g0, q0, kv0)) break;
         for (int kb = 0; kb < nb && ok; ++kb) {
-            const int s = n_load & 1;
-            const uint32_t qq = smem_u32(sm.q(s)), vv = smem_u32(sm.v(s));
-            ok = mbar_wait(&bars[B_P_READY], n_p++ & 1, sm.abort, p.hdr) &&
-                 mbar_wait(&bars[B_O_EMPTY], (n_o++ & 1) ^ 1, sm.abort, p.hdr);
+            const uint32_t gg = g0 + kb;
+            const int sq = (q0 + kb) & 1, skv = (kv0 + kb) & 1;
+            // MMA4: this block's DS, once E_V has decayed its values and E_S
+            // has read the previous DS.
+            ok = mbar_wait(&bars[B_VH_READY], n_vh & 1, sm.abort, p.hdr) &&
+                 mbar_wait(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr);
+            if (!ok) break;
+            ++n_vh;
+            tc_fence_after();
+            mma4(skv, false);
+            mma_commit(&bars[B_DS_FULL]);
+            mma_commit(&bars[B_VH_FREE]);
+            mma_commit(&bars[B_KE0 + skv]);
+            ++n_ds;
+            // MMA3: OE[g & 1] = Q S_in (hi and lo), once E_S has written the copy.
+            ok = mbar_wait(&bars[B_S_READY], n_s & 1, sm.abort, p.hdr);
+            if (!ok) break;
+            ++n_s;
+            tc_fence_after();
+            {
+                const uint32_t qq = smem_u32(sm.q(sq));
+                const uint32_t d = tmem + COL_OE + (uint32_t)DV * (gg & 1);
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ss(d, desc_kmajor(qq, ks), desc_mn64(part ? slo : shi, ks),
+                               IDESC_QS, (part || ks) ? 1u : 0u);
+            }
+            mma_commit(&bars[B_S_FREE]);
+            mma_commit(&bars[B_QE0 + sq]);
+            // MMA1 of the next block, so that E_P overlaps this block's MMA2.
+            if (kb + 1 < nb && !(ok = mma1(gg + 1, q0 + kb + 1, kv0 + kb + 1))) break;
+            // MMA2: OI = P V (P hi and lo from TMEM), once E_P is done and
+            // E_O has read the previous OI.
+            ok = mbar_wait(&bars[B_P_READY0 + (gg & 1)], (gg >> 1) & 1, sm.abort, p.hdr) &&
+                 mbar_wait(&bars[B_O_EMPTY], (gg & 1) ^ 1, sm.abort, p.hdr);
             if (!ok) break;
             tc_fence_after();
+            {
+                const uint32_t vv = smem_u32(sm.v(skv));
+                const uint32_t a = tmem + COL_SP + 128u * (gg & 1);
+                // K-step ks (tokens 16ks..16ks+15) sits in chunk ks/2: hi words
+                // at column 32(ks/2) + 8(ks%2), lo words 16 columns further.
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_ts(tmem + COL_OI, tmem + COL_SB + ks * 8, desc_mnmajor(vv, ks), IDESC_PV,
-                       ks > 0 ? 1u : 0u);
-            mma_commit(&bars[B_SB_FREE]);
-            ok = mbar_wait(&bars[B_S_READY], n_s++ & 1, sm.abort, p.hdr);
-            if (!ok) break;
-            tc_fence_after();
+                for (int part = 0; part < 2; ++part)
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_ss(tmem + COL_OE, desc_kmajor(qq, ks), desc_kmajor(s16, ks), IDESC_QS,
-                       ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ts(tmem + COL_OI, a + 32u * (ks >> 1) + 8u * (ks & 1) + 16u * part,
+                               desc_mn64(vv, ks), IDESC_PV, (part || ks) ? 1u : 0u);
+            }
             mma_commit(&bars[B_O_FULL]);
-            // MMA4 of this block, then MMA1 of the next (its tiles are converted
-            // while this block's epilogues run).
-            if (!(ok = issue_vk(s))) break;
-            if (kb + 1 < nb && !(ok = issue_qk(n_load + 1))) break;
-            ++n_load;
+            mma_commit(&bars[B_VE0 + skv]);
         }
         if (!ok) break;
+        nq += nb;
+        nkv += nb;
+        g += nb;
     }
     // Make sure no MMA is in flight before TMEM is released.
     mma_commit(&bars[B_FIN]);
@@ -705,239 +704,51 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
     mbar_wait(&bars[B_FIN], 0, &never, p.hdr, DRAIN_LIMIT_NS);
 }
 
-// Row r of a 16-bit tile as 64 packed words (two elements each).
-__device__ __forceinline__ void load_row_packed(const uint8_t* tile, int r, uint32_t (&w)[64])
-{
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        const uint4 x = *reinterpret_cast<const uint4*>(tile + chunk_off(r, c));
-        w[4 * c + 0] = x.x;
-        w[4 * c + 1] = x.y;
-        w[4 * c + 2] = x.z;
-        w[4 * c + 3] = x.w;
-    }
-}
-
-__device__ __forceinline__ float absmax_bf16_packed(const uint32_t (&w)[64])
-{
-    float m = 0.f;
-#pragma unroll
-    for (int i = 0; i < 64; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[i])), fabsf(bf16_hi(w[i]))));
-    return m;
-}
-
-// Store packed bf16 words times f as fp16 into row r.
-__device__ __forceinline__ void store_bf16_packed_as_f16(uint8_t* tile, int r,
-                                                         const uint32_t (&w)[64], float f)
-{
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-        uint4 x;
-        x.x = pack_f16x2(bf16_lo(w[4 * c + 0]) * f, bf16_hi(w[4 * c + 0]) * f);
-        x.y = pack_f16x2(bf16_lo(w[4 * c + 1]) * f, bf16_hi(w[4 * c + 1]) * f);
-        x.z = pack_f16x2(bf16_lo(w[4 * c + 2]) * f, bf16_hi(w[4 * c + 2]) * f);
-        x.w = pack_f16x2(bf16_lo(w[4 * c + 3]) * f, bf16_hi(w[4 * c + 3]) * f);
-        *reinterpret_cast<uint4*>(tile + chunk_off(r, c)) = x;
-    }
-}
-
-// Max |x| of row r of a bf16 tile (streaming, few registers). With the sign
-// bit cleared, bf16 bit patterns order like their magnitudes, so the maximum
-// is a packed unsigned 16-bit maximum.
-__device__ __forceinline__ float row_absmax_bf16(const uint8_t* tile, int r)
-{
-    uint32_t m = 0u;
-#pragma unroll 4
-    for (int c = 0; c < 16; ++c) {
-        const uint4 x = *reinterpret_cast<const uint4*>(tile + chunk_off(r, c));
-        m = __vmaxu2(m, __vmaxu2(__vmaxu2(x.x & 0x7fff7fffu, x.y & 0x7fff7fffu),
-                                 __vmaxu2(x.z & 0x7fff7fffu, x.w & 0x7fff7fffu)));
-    }
-    return fmaxf(bf16_lo(m), bf16_hi(m));
-}
-
-// Rewrite row r of a bf16 tile in place as fp16 times f (streaming).
-__device__ __forceinline__ void row_bf16_to_f16(uint8_t* tile, int r, float f)
-{
-#pragma unroll 4
-    for (int c = 0; c < 16; ++c) {
-        uint4* ptr = reinterpret_cast<uint4*>(tile + chunk_off(r, c));
-        const uint4 x = *ptr;
-        *ptr = make_uint4(pack_f16x2(bf16_lo(x.x) * f, bf16_hi(x.x) * f),
-                          pack_f16x2(bf16_lo(x.y) * f, bf16_hi(x.y) * f),
-                          pack_f16x2(bf16_lo(x.z) * f, bf16_hi(x.z) * f),
-                          pack_f16x2(bf16_lo(x.w) * f, bf16_hi(x.w) * f));
-    }
-}
-
-// Q converters (the two spare warps of the control warpgroup): fp16 Q with
-// one power-of-two scale per row, for phase-C blocks, in parallel with the K
-// and V converters. Thread t owns rows t and t + 64.
-__device__ void qcv_role(const Params& p, const Smem& sm, int warp, int lane)
-{
-    uint64_t* bars = sm.bars;
-    const int t = ((warp & 1) << 5) | lane;
-    uint32_t n_load = 0, n_q[2] = {0, 0};
-    for (uint32_t k = 0;; ++k) {
-        const int slot = k & 1;
-        if (!wait_warp(&bars[B_ITEM_FULL0 + slot], (k >> 1) & 1, sm.abort, p.hdr)) break;
-        const Item it = sm.ring[slot];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_ITEM_EMPTY0 + slot]);
-        if (!it.valid) break;
-        const int nb = num_blocks(it.len);
-        bool ok = true;
-        for (int pass = it.p_ord < it.nseg - 1 ? 0 : 1; pass < 2 && ok; ++pass) {
-            for (int kb = 0; kb < nb && ok; ++kb) {
-                const int s = n_load & 1;
-                const int sl = n_load & 3;
-                ok = wait_warp(&bars[B_SC_EMPTY0 + sl], ((n_load >> 2) & 1) ^ 1, sm.abort, p.hdr);
-                if (!ok) break;
-                if (pass == 1) {
-                    ok = wait_warp(&bars[B_QFULL0 + s], n_q[s]++ & 1, sm.abort, p.hdr);
-                    if (!ok) break;
-#pragma unroll 1
-                    for (int h = 0; h < 2; ++h) {
-                        const int r = t + 64 * h;
-                        const Pow2 qs = pow2_for(row_absmax_bf16(sm.q(s), r));
-                        row_bf16_to_f16(sm.q(s), r, qs.down);
-                        sm.sc[sl].qe[r] = qs.ue;
-                    }
-                    fence_proxy_async();
-                    mbar_arrive(&bars[B_CONV0 + s]);
-                }
-                mbar_arrive(&bars[B_SC_FULL0 + sl]);
-                ++n_load;
-            }
-        }
-        if (!ok) break;
-    }
-}
-
-// Converter group: fp16 operands for the tensor cores as soon as a block's
-// tiles land. Thread r owns row r of each tile. Q rows get their own
-// power-of-two scale; K and V get one scale per tile (a maximum over the
-// group). Phase-A blocks only need the decayed keys and V. The scales go to
-// the OS group through the ScaleRec ring.
-__device__ void cv_role(const Params& p, const Smem& sm, int warp, int lane)
-{
-    uint64_t* bars = sm.bars;
-    const int r = ((warp & 3) << 5) | lane;
-    const int w = warp & 3;
-    const int rev = p.reverse;
-    uint32_t n_load = 0, n_sync = 0;
-
-    // Tile maxima of (a, b) over the 128 rows.
-    auto tile_max2 = [&](float& a, float& b) -> bool {
-        a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a)));
-        b = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(b)));
-        float* red = sm.red + (n_load & 1) * 8;
-        if (lane == 0) {
-            red[w] = a;
-            red[4 + w] = b;
-        }
-        if (!group_sync(&bars[B_CV_SYNC], n_sync, sm.abort, p.hdr)) return false;
-        a = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-        b = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
-        return true;
-    };
-
-    for (uint32_t k = 0;; ++k) {
-        const int slot = k & 1;
-        if (!wait_warp(&bars[B_ITEM_FULL0 + slot], (k >> 1) & 1, sm.abort, p.hdr)) break;
-        const Item it = sm.ring[slot];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_ITEM_EMPTY0 + slot]);
-        if (!it.valid) break;
-        const float slope = p.slopes[it.head];
-        const int nb = num_blocks(it.len);
-        const bool has_succ = it.p_ord < it.nseg - 1;
-        bool ok = true;
-        for (int pass = has_succ ? 0 : 1; pass < 2 && ok; ++pass) {
-            for (int kb = 0; kb < nb && ok; ++kb) {
-                const int s = n_load & 1;
-                const int L = min(C, it.len - block_t0(it.len, kb, rev));
-                const int sl = n_load & 3;
-                ScaleRec* rec = sm.sc + sl;
-                ok = wait_warp(&bars[B_FULL0 + s], (n_load >> 1) & 1, sm.abort, p.hdr) &&
-                     wait_warp(&bars[B_SC_EMPTY0 + sl], ((n_load >> 2) & 1) ^ 1, sm.abort, p.hdr);
-                if (!ok) break;
-                const bool live = r < L;
-                // K (phase A: already decayed) and V: one scale per tile.
-                const float kf = pass == 0
-                                     ? (live ? expf(-slope * (float)(rev ? r : L - 1 - r)) : 0.f)
-                                     : (live ? 1.f : 0.f);
-                float km = row_absmax_bf16(sm.k(s), r) * kf;
-                float vm = live ? row_absmax_bf16(sm.v(s), r) : 0.f;
-                if (!(ok = tile_max2(km, vm))) break;
-                const Pow2 ks = pow2_for(km), vs = pow2_for(vm);
-                row_bf16_to_f16(sm.v(s), r, live ? vs.down : 0.f);
-                row_bf16_to_f16(sm.k(s), r, kf * ks.down);
-                if (r == 0) {
-                    rec->kc = ks.ue;
-                    rec->vc = vs.ue;
-                }
-                fence_proxy_async();
-                mbar_arrive(&bars[pass == 0 ? B_KT0 + s : B_CONV0 + s]);
-                mbar_arrive(&bars[B_SC_FULL0 + sl]);
-                ++n_load;
-            }
-        }
-        if (!ok) break;
-    }
-}
-
-// PE group: after Q K^T, the decayed causal mask (fp16 P into TMEM, in place
-// over the scores) and the decayed keys for the state update (in place over
-// K). Thread i owns TMEM lane / tile row i.
+// P group: E_P for every phase-C block.
 template <int REV>
-__device__ void pe_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
+__device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
     uint64_t* bars = sm.bars;
     const int w = warp & 3;
     const int row = (w << 5) | lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(w << 5) << 16);
-    float* pw = sm.pw_pe;
-    uint32_t n_load = 0, n_sblk = 0, n_sync = 0;
+    float* pw = sm.pw;
+    uint32_t g = 0, n_sync = 0;
+    Item it;
     for (uint32_t k = 0;; ++k) {
-        const int slot = k & 1;
-        if (!wait_warp(&bars[B_ITEM_FULL0 + slot], (k >> 1) & 1, sm.abort, p.hdr)) break;
-        const Item it = sm.ring[slot];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_ITEM_EMPTY0 + slot]);
-        if (!it.valid) break;
+        if (!next_item(p, sm, k, it, true, lane)) break;
         const float slope = p.slopes[it.head];
-        if (!group_sync(&bars[B_PE_SYNC], n_sync, sm.abort, p.hdr)) break;
+        if (!group_sync(&bars[B_P_SYNC], n_sync, sm.abort, p.hdr)) break;
         pw[row] = expf(-slope * (float)row);
         if (row == 0) pw[C] = expf(-slope * (float)C);
-        if (!group_sync(&bars[B_PE_SYNC], n_sync, sm.abort, p.hdr)) break;
+        if (!group_sync(&bars[B_P_SYNC], n_sync, sm.abort, p.hdr)) break;
         const int nb = num_blocks(it.len);
-        if (it.p_ord < it.nseg - 1) n_load += nb;  // phase A blocks need no PE work
         bool ok = true;
-        for (int kb = 0; kb < nb && ok; ++kb) {
-            const int s = n_load & 1;
+        for (int kb = 0; kb < nb && ok; ++kb, ++g) {
             const int L = min(C, it.len - block_t0(it.len, kb, REV));
-            ok = wait_warp(&bars[B_SBLK_FULL], n_sblk++ & 1, sm.abort, p.hdr);
+            const int buf = g & 1;
+            ok = wait_warp(&bars[B_SP_FULL0 + buf], (g >> 1) & 1, sm.abort, p.hdr);
             if (!ok) break;
             tc_fence_after();
-            // E_P. Chunk c covers columns 32c..32c+31; warp w holds rows
-            // 32w..32w+31, so chunks before (forward) / after (reverse) the
-            // diagonal chunk are fully causal and the rest fully masked.
+            const uint32_t base = lane_addr + COL_SP + 128u * buf;
+            // Chunk c covers columns 32c..32c+31; warp w holds rows 32w..32w+31,
+            // so chunks before (forward) / after (reverse) the diagonal chunk
+            // are fully causal and the rest fully masked.
             const bool row_live = REV ? true : row < L;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                uint32_t pk[16];
+                uint32_t hi[16], lo[16];
                 const bool active = REV ? (c >= w) : (c <= w);
                 if (active) {
                     uint32_t r32[32];
-                    tmem_ld32(lane_addr + COL_SB + 32 * c, r32);
+                    tmem_ld32(base + 32 * c, r32);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
+                    for (int e = 0; e < 16; ++e) {
                         float x2[2];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
-                            const int j = 32 * c + e + u;
+                            const int j = 32 * c + 2 * e + u;
                             bool keep;
                             int m;
                             if (REV) {
@@ -947,124 +758,182 @@ __device__ void pe_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
                                 keep = (c < w || j <= row) && row_live;
                                 m = row - j;
                             }
-                            x2[u] = keep ? __uint_as_float(r32[e + u]) * pw[keep ? m : 0] : 0.f;
+                            x2[u] = keep ? __uint_as_float(r32[2 * e + u]) * pw[keep ? m : 0] : 0.f;
                         }
-                        pk[e >> 1] = pack_f16x2(x2[0], x2[1]);
+                        split2(x2[0], x2[1], hi[e], lo[e]);
                     }
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
                 }
-                tmem_st16(lane_addr + COL_SB + 16 * c, pk);
+                tmem_st16(base + 32 * c, hi);
+                tmem_st16(base + 32 * c + 16, lo);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars[B_P_READY]);
-            // E_K: decayed keys lam^(L-1-j) k_j (reverse: lam^j), in place (fp16).
-            {
-                const float f = row < L ? pw[REV ? row : L - 1 - row] : 0.f;
-                uint8_t* kt = sm.k(s);
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    uint4* ptr = reinterpret_cast<uint4*>(kt + chunk_off(row, c));
-                    uint4 x = *ptr;
-                    uint32_t* e4 = reinterpret_cast<uint32_t*>(&x);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&e4[u]));
-                        e4[u] = pack_f16x2(h.x * f, h.y * f);
-                    }
-                    *ptr = x;
-                }
-            }
-            fence_proxy_async();
-            mbar_arrive(&bars[B_KT0 + s]);
-            ++n_load;
+            mbar_arrive(&bars[B_P_READY0 + buf]);
         }
         if (!ok) break;
     }
 }
 
-// OS group: S = lam^L S + up * DS for the next DS use (phase A or C).
-__device__ __forceinline__ bool os_accumulate_ds(const Params& p, const Smem& sm,
-                                                 uint32_t lane_addr, float (&S)[D], int L,
-                                                 float slope, float up, uint32_t& n_ds)
-{
-    if (!wait_warp(&sm.bars[B_DS_FULL], n_ds & 1, sm.abort, p.hdr)) return false;
-    tc_fence_after();
-    const float dL = expf(-slope * (float)L);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_addr + COL_DS + 32 * c, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 32; ++x)
-            S[32 * c + x] = fmaf(dL, S[32 * c + x], up * __uint_as_float(r[x]));
-    }
-    tc_fence_before();
-    mbar_arrive(&sm.bars[B_DS_EMPTY]);
-    mbar_arrive(&sm.bars[B_SC_EMPTY0 + (n_ds & 3)]);
-    ++n_ds;
-    return true;
-}
-
-// OS group: fp16 copy of the state for MMA3 (row a of S^T). One power-of-two
-// scale per 32 state columns (one warp), from a warp-wide maximum.
-__device__ __forceinline__ void os_publish_s16(const Smem& sm, int a, const float (&S)[D], int par)
-{
-    const float m = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(row_absmax(S))));
-    const Pow2 sc = pow2_for(m);
-    store_row_f16(sm.s16(), a, S, sc.down);
-    if ((a & 31) == 0) sm.hs[par * 4 + (a >> 5)] = sc.ue;
-    fence_proxy_async();
-    mbar_arrive(&sm.bars[B_S_READY]);
-}
-
+// VO group: E_V (decayed values, hi and lo, for every block) and E_O (the
+// output rows of every phase-C block).
 template <int REV, int OUT_F32>
-__device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
+__device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
     uint64_t* bars = sm.bars;
-    const int a = ((warp & 3) << 5) | lane;  // TMEM lane: output row i / state column a
-    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) << 5) << 16);
-    float slope = 0.f;
-    // n_blk counts phase-C blocks (one o_full and s_ready phase each);
-    // n_ds counts DS uses (= blocks loaded = scale records).
-    uint32_t n_sync = 0, n_blk = 0, n_ds = 0;
-    float S[D];  // column a of the fp32 state: S[x] = state[x][a]
-
+    const int w = warp & 3;
+    const int row = (w << 5) | lane;  // E_V: token row of the V tile; E_O: output row
+    const uint32_t lane_addr = tmem + ((uint32_t)(w << 5) << 16);
+    uint32_t nkv = 0, n_vh = 0, g = 0;
+    Item it;
+    // E_V for the block at segment offset t0 with L valid tokens; the value
+    // of token j is scaled by lam^m(j) (0 for j >= L).
+    auto e_v = [&](float slope, int L, int m) -> bool {
+        const int s = nkv & 1;
+        if (!wait_warp(&bars[B_VF0 + s], (nkv >> 1) & 1, sm.abort, p.hdr)) return false;
+        if (!wait_warp(&bars[B_VH_FREE], (n_vh & 1) ^ 1, sm.abort, p.hdr)) return false;
+        const float f = row < L ? expf(-slope * (float)m) : 0.f;
+        const uint8_t* src = sm.v(s);
+        float x[DV];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 u = *reinterpret_cast<const uint4*>(src + swz(row, c));
+            x[8 * c + 0] = bf16_lo(u.x) * f; x[8 * c + 1] = bf16_hi(u.x) * f;
+            x[8 * c + 2] = bf16_lo(u.y) * f; x[8 * c + 3] = bf16_hi(u.y) * f;
+            x[8 * c + 4] = bf16_lo(u.z) * f; x[8 * c + 5] = bf16_hi(u.z) * f;
+            x[8 * c + 6] = bf16_lo(u.w) * f; x[8 * c + 7] = bf16_hi(u.w) * f;
+        }
+        store_split_row(sm.vh(), sm.vl(), row, x);
+        fence_proxy_async();
+        mbar_arrive(&bars[B_VH_READY]);
+        ++nkv;
+        ++n_vh;
+        return true;
+    };
     for (uint32_t k = 0;; ++k) {
-        const int slot = k & 1;
-        if (!wait_warp(&bars[B_ITEM_FULL0 + slot], (k >> 1) & 1, sm.abort, p.hdr)) break;
-        const Item it = sm.ring[slot];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[B_ITEM_EMPTY0 + slot]);
-        if (!it.valid) break;
-        slope = p.slopes[it.head];
+        if (!next_item(p, sm, k, it, true, lane)) break;
+        const float slope = p.slopes[it.head];
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
-
-#pragma unroll
-        for (int x = 0; x < D; ++x) S[x] = 0.f;
         if (has_succ) {
-            // Phase A: local state of the segment.
             for (int kb = 0; kb < nb && ok; ++kb) {
-                const int L = min(C, it.len - block_t0(it.len, kb, REV));
-                const ScaleRec* rec = sm.sc + (n_ds & 3);
-                ok = wait_warp(&bars[B_SC_FULL0 + (n_ds & 3)], (n_ds >> 2) & 1, sm.abort, p.hdr);
-                if (!ok) break;
-                const float up = up_of(rec->kc) * up_of(rec->vc);
-                ok = os_accumulate_ds(p, sm, lane_addr, S, L, slope, up, n_ds);
+                const int t0 = block_t0(it.len, kb, REV);
+                const int L = min(C, it.len - t0);
+                ok = e_v(slope, L, REV ? t0 + row : it.len - 1 - (t0 + row));
             }
             if (!ok) break;
         }
+        auto e_v_c = [&](int kb) -> bool {
+            const int L = min(C, it.len - block_t0(it.len, kb, REV));
+            return e_v(slope, L, REV ? row : L - 1 - row);
+        };
+        if (!e_v_c(0)) break;
+        for (int kb = 0; kb < nb && ok; ++kb, ++g) {
+            if (kb + 1 < nb && !(ok = e_v_c(kb + 1))) break;
+            // E_O: O = OI + lam^(i+1) OE (reverse: lam^(L-i)).
+            ok = wait_warp(&bars[B_O_FULL], g & 1, sm.abort, p.hdr);
+            if (!ok) break;
+            tc_fence_after();
+            const int t0 = block_t0(it.len, kb, REV);
+            const int L = min(C, it.len - t0);
+            const float rowc = expf(-slope * (float)(REV ? max(L - row, 0) : row + 1));
+            const bool store = row < L;
+            const long long orow = it.out_row0 + t0 + row;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t ri[32], re[32];
+                tmem_ld32(lane_addr + COL_OI + 32 * h, ri);
+                tmem_ld32(lane_addr + COL_OE + (uint32_t)DV * (g & 1) + 32 * h, re);
+                tmem_wait_ld();
+                float ov[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x)
+                    ov[x] = fmaf(rowc, __uint_as_float(re[x]), __uint_as_float(ri[x]));
+                if (store) {
+                    const size_t off = (size_t)orow * D + DV * it.half + 32 * h;
+                    if (OUT_F32) {
+                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + off);
+#pragma unroll
+                        for (int x = 0; x < 8; ++x)
+                            dst[x] = make_float4(ov[4 * x], ov[4 * x + 1], ov[4 * x + 2], ov[4 * x + 3]);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x)
+                            dst[x] = make_uint4(pack_bf16x2(ov[8 * x + 0], ov[8 * x + 1]),
+                                                pack_bf16x2(ov[8 * x + 2], ov[8 * x + 3]),
+                                                pack_bf16x2(ov[8 * x + 4], ov[8 * x + 5]),
+                                                pack_bf16x2(ov[8 * x + 6], ov[8 * x + 7]));
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[B_O_EMPTY]);
+        }
+        if (!ok) break;
+    }
+}
+
+// S group: E_S (the fp32 state, row a of this item's 128 x 64 state per
+// thread), the hi/lo state copies for MMA3, and the scan between segments.
+template <int REV>
+__device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
+{
+    uint64_t* bars = sm.bars;
+    const int a = ((warp & 3) << 5) | lane;  // TMEM lane = key dim a
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) << 5) << 16);
+    uint32_t n_ds = 0, n_s = 0, n_sync = 0;
+    float S[DV];
+    Item it;
+    // DS row a -> x (with S = dL * S + DS when accumulate).
+    auto read_ds = [&](float dL, bool accumulate) -> bool {
+        if (!wait_warp(&bars[B_DS_FULL], n_ds & 1, sm.abort, p.hdr)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+            tmem_ld32(lane_addr + COL_DS + 32 * h, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+                S[32 * h + x] = accumulate ? fmaf(dL, S[32 * h + x], __uint_as_float(r[x]))
+                                           : __uint_as_float(r[x]);
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[B_DS_EMPTY]);
+        ++n_ds;
+        return true;
+    };
+    // Hi/lo copies of the state for the next MMA3.
+    auto publish_copy = [&]() -> bool {
+        if (!wait_warp(&bars[B_S_FREE], (n_s & 1) ^ 1, sm.abort, p.hdr)) return false;
+        store_split_row(sm.sh(), sm.sl(), a, S);
+        fence_proxy_async();
+        mbar_arrive(&bars[B_S_READY]);
+        ++n_s;
+        return true;
+    };
+    for (uint32_t k = 0;; ++k) {
+        if (!next_item(p, sm, k, it, true, lane)) break;
+        const float slope = p.slopes[it.head];
+        const int nb = num_blocks(it.len);
+        const bool has_succ = it.p_ord < it.nseg - 1;
+        const int chain2 = 2 * it.chain + it.half;
+        bool ok = true;
+        if (has_succ) {
+            if (!read_ds(0.f, false)) break;  // S = S_loc
+        } else {
+#pragma unroll
+            for (int x = 0; x < DV; ++x) S[x] = 0.f;
+        }
         // Incoming state: the predecessor's inclusive prefix (zero for the first segment).
-        const float* src = p.incl + ((size_t)it.chain * 2 + ((it.p_ord - 1) & 1)) * D * D +
-                           (size_t)a * D;
+        const float* src = p.incl + (((size_t)chain2 * 2 + ((it.p_ord - 1) & 1)) * D + a) * DV;
         if (it.p_ord > 0) {
             if (a == 0) {
-                const int* flag = p.chain_flags + it.chain;
+                const int* flag = p.chain_flags + chain2;
                 const unsigned long long t0 = globaltimer();
                 int seen;
                 for (uint32_t spin = 0;; ++spin) {
@@ -1080,17 +949,16 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
                     __nanosleep(128);
                 }
             }
-            if (!group_sync(&bars[B_OS_SYNC], n_sync, sm.abort, p.hdr)) break;
+            if (!group_sync(&bars[B_S_SYNC], n_sync, sm.abort, p.hdr)) break;
         }
         {
-            // S_prev = the predecessor's inclusive prefix (0 for the first
-            // segment). With a successor, publish lam^len S_prev + S_loc.
-            // Phase C continues from S_prev.
+            // S_prev = the predecessor's prefix; with a successor, publish
+            // lam^len S_prev + S_loc. Phase C continues from S_prev.
             const float dl = expf(-slope * (float)it.len);
-            float* dst = p.incl + ((size_t)it.chain * 2 + (it.p_ord & 1)) * D * D + (size_t)a * D;
+            float* dst = p.incl + (((size_t)chain2 * 2 + (it.p_ord & 1)) * D + a) * DV;
             const bool has_prev = it.p_ord > 0;
 #pragma unroll
-            for (int x = 0; x < D / 4; ++x) {
+            for (int x = 0; x < DV / 4; ++x) {
                 const float4 w = has_prev ? ld_cg_ordered(src + 4 * x) : make_float4(0.f, 0.f, 0.f, 0.f);
                 if (has_succ)
                     st_cg_ordered(dst + 4 * x,
@@ -1104,92 +972,39 @@ __device__ void os_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         }
         if (has_succ) {
             __threadfence();
-            if (!group_sync(&bars[B_OS_SYNC], n_sync, sm.abort, p.hdr)) break;
+            if (!group_sync(&bars[B_S_SYNC], n_sync, sm.abort, p.hdr)) break;
             if (a == 0 && !p.skip_publish) {
-                int* flag = p.chain_flags + it.chain;
+                int* flag = p.chain_flags + chain2;
                 asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(it.p_ord + 1) : "memory");
             }
         }
-        os_publish_s16(sm, a, S, n_blk & 1);
-
+        if (!publish_copy()) break;
         for (int kb = 0; kb < nb && ok; ++kb) {
-            const int par = n_blk & 1;
-            const int t0 = block_t0(it.len, kb, REV);
-            const int L = min(C, it.len - t0);
-            const ScaleRec* rec = sm.sc + (n_ds & 3);
-            // E_O: O = up_Q up_K up_V * OI + lam^(i+1) * up_Q * up_S[col] * OE
-            // (reverse: lam^(L-i)).
-            ok = wait_warp(&bars[B_O_FULL], n_blk & 1, sm.abort, p.hdr) &&
-                 wait_warp(&bars[B_S_READY], n_blk & 1, sm.abort, p.hdr) &&
-                 wait_warp(&bars[B_SC_FULL0 + (n_ds & 3)], (n_ds >> 2) & 1, sm.abort, p.hdr);
-            if (!ok) break;
-            tc_fence_after();
-            const float up_kv = up_of(rec->kc) * up_of(rec->vc);
-            const float up_q = up_of(rec->qe[a]);
-            const float gi = up_q * up_kv;
-            const float rowc = expf(-slope * (float)(REV ? max(L - a, 0) : a + 1)) * up_q;
-            const uint8_t* hsp = sm.hs + par * 4;
-            const bool store = a < L;
-            const long long orow = it.out_row0 + t0 + a;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t ri[16], re[16];
-                tmem_ld16(lane_addr + COL_OI + 16 * c, ri);
-                tmem_ld16(lane_addr + COL_OE + 16 * c, re);
-                tmem_wait_ld();
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    float ov[8];
-                    const float ec = rowc * up_of(hsp[c >> 1]);
-#pragma unroll
-                    for (int x = 0; x < 8; ++x)
-                        ov[x] = fmaf(ec, __uint_as_float(re[8 * h + x]), gi * __uint_as_float(ri[8 * h + x]));
-                    if (store) {
-                        if (OUT_F32) {
-                            float4* dst = reinterpret_cast<float4*>(
-                                static_cast<float*>(p.o) + orow * D + 16 * c + 8 * h);
-                            dst[0] = make_float4(ov[0], ov[1], ov[2], ov[3]);
-                            dst[1] = make_float4(ov[4], ov[5], ov[6], ov[7]);
-                        } else {
-                            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + orow * D +
-                                                      16 * c + 8 * h) =
-                                make_uint4(pack_bf16x2(ov[0], ov[1]), pack_bf16x2(ov[2], ov[3]),
-                                           pack_bf16x2(ov[4], ov[5]), pack_bf16x2(ov[6], ov[7]));
-                        }
-                    }
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&bars[B_O_EMPTY]);
-            // E_S.
-            if (!(ok = os_accumulate_ds(p, sm, lane_addr, S, L, slope, up_kv, n_ds))) break;
-            if (kb + 1 < nb) os_publish_s16(sm, a, S, (n_blk + 1) & 1);
-            ++n_blk;
+            const int L = min(C, it.len - block_t0(it.len, kb, REV));
+            if (!(ok = read_ds(expf(-slope * (float)L), true))) break;
+            if (kb + 1 < nb && !(ok = publish_copy())) break;
         }
         if (!ok) break;
         if (it.p_ord == it.nseg - 1 && p.state_out) {
-            float* dst = p.state_out + (size_t)it.chain * D * D + a;
+            float4* dst = reinterpret_cast<float4*>(p.state_out + ((size_t)it.chain * D + a) * D +
+                                                    DV * it.half);
 #pragma unroll
-            for (int x = 0; x < D; ++x) dst[(size_t)x * D] = S[x];
+            for (int x = 0; x < DV / 4; ++x)
+                dst[x] = make_float4(S[4 * x], S[4 * x + 1], S[4 * x + 2], S[4 * x + 3]);
         }
     }
 }
 
 // Small shared state at the start of the dynamic region; the 1024-aligned
 // tile region follows (SMEM_BYTES reserves the worst-case alignment gap).
-constexpr uint32_t SM_BARS = 0;                       // 36 x 8 B
-constexpr uint32_t SM_RING = 288;                     // 2 x Item
-constexpr uint32_t SM_PW = 384;                       // (C+1) floats
-constexpr uint32_t SM_SC = 912;                       // 4 x ScaleRec (144 B)
-constexpr uint32_t SM_RED = SM_SC + 4 * 144;          // 16 floats
-constexpr uint32_t SM_HS = SM_RED + 64;               // [2][128] bytes
-constexpr uint32_t SM_TMEM = SM_HS + 256;             // u32
+constexpr uint32_t SM_BARS = 0;                       // NUM_BARS x 8 B
+constexpr uint32_t SM_RING = 256;                     // 2 x Item
+constexpr uint32_t SM_PW = 384;                       // (C + 1) floats
+constexpr uint32_t SM_TMEM = SM_PW + 4 * (C + 4);     // u32
 constexpr uint32_t SM_ABORT = SM_TMEM + 4;            // int
 constexpr uint32_t SM_SMALL = SM_ABORT + 4;
-static_assert(NUM_BARS <= 36, "barrier area");
+static_assert(NUM_BARS * 8 <= SM_RING, "barrier area");
 static_assert(sizeof(Item) * 2 <= SM_PW - SM_RING, "ring area");
-static_assert(SM_PW + (C + 1) * 4 <= SM_SC, "pw area");
-static_assert(sizeof(ScaleRec) == 144, "scale record");
 constexpr uint32_t SMEM_BYTES = SM_SMALL + 1023 + SMEM_TILES;
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
@@ -1209,24 +1024,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     sm.bars = bars;
     sm.ring = reinterpret_cast<Item*>(dsmem + SM_RING);
     sm.abort = abort_flag;
-    sm.pw_pe = reinterpret_cast<float*>(dsmem + SM_PW);
-    sm.sc = reinterpret_cast<ScaleRec*>(dsmem + SM_SC);
-    sm.red = reinterpret_cast<float*>(dsmem + SM_RED);
-    sm.hs = dsmem + SM_HS;
+    sm.pw = reinterpret_cast<float*>(dsmem + SM_PW);
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
-        uint32_t counts[NUM_BARS];
-        for (int i = 0; i < NUM_BARS; ++i) counts[i] = 128;
-        counts[B_FULL0] = counts[B_FULL1] = counts[B_EMPTY0] = counts[B_EMPTY1] = 1;
-        counts[B_SBLK_FULL] = counts[B_SB_FREE] = counts[B_O_FULL] = counts[B_DS_FULL] = 1;
-        counts[B_ITEM_FULL0] = counts[B_ITEM_FULL1] = counts[B_FIN] = 1;
-        counts[B_QFULL0] = counts[B_QFULL1] = 1;
-        counts[B_ITEM_EMPTY0] = counts[B_ITEM_EMPTY1] = 15;  // MMA lane + 14 group warps
-        // Q converters (64 threads) join the K/V converters (128).
-        counts[B_CONV0] = counts[B_CONV1] = 192;
-        counts[B_SC_FULL0] = counts[B_SC_FULL1] = counts[B_SC_FULL2] = counts[B_SC_FULL3] = 192;
-        for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], counts[i]);
+        for (int i = 0; i < NUM_BARS; ++i) {
+            uint32_t count = 1;  // TMA expect_tx arrivals, MMA commits, single threads
+            if (i == B_P_READY0 || i == B_P_READY1 || i == B_VH_READY || i == B_DS_EMPTY ||
+                i == B_S_READY || i == B_O_EMPTY || i == B_P_SYNC || i == B_S_SYNC)
+                count = 128;
+            if (i == B_ITEM_EMPTY0 || i == B_ITEM_EMPTY1) count = 1 + 12;  // MMA lane + 12 group warps
+            mbar_init(&bars[i], count);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tq)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tk)) : "memory");
@@ -1247,16 +1056,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_CTRL));
         if (warp == 0 && lane == 0) producer_role(p, &tq, &tk, &tv, sm);
         if (warp == 1 && lane == 0) mma_role(p, sm, tmem);
-        if (warp >= 2) qcv_role(p, sm, warp, lane);
     } else if (warp < 8) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_CV));
-        cv_role(p, sm, warp, lane);
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_P));
+        p_role<REV>(p, sm, tmem, warp, lane);
     } else if (warp < 12) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PE));
-        pe_role<REV>(p, sm, tmem, warp, lane);
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_VO));
+        vo_role<REV, OUT_F32>(p, sm, tmem, warp, lane);
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_OS));
-        os_role<REV, OUT_F32>(p, sm, tmem, warp, lane);
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_S));
+        s_role<REV>(p, sm, tmem, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -1376,31 +1184,34 @@ static int num_sms()
     return n;
 }
 
-// Segment length: the tuning value, or the candidate among 1K..8K tokens
-// that minimises (rounds of persistent CTAs) x (blocks per item + fixed
-// per-item cost), with phase A counted for items that have a successor.
+// Segment length: the tuning value, or the candidate (powers of two from 1K
+// tokens up to one segment per chain) that minimises (rounds of persistent
+// CTAs) x (blocks per item + a fixed per-item cost), with phase A counted
+// for items that have a successor. Independent of the device, so that the
+// workspace size depends only on the arguments.
 static int choose_seg(const Problems& P, int seg_tuning, bool varlen)
 {
     if (seg_tuning > 0) return seg_tuning;
-    if (varlen) return 2048;
-    const long long N = P.N, chains = P.count();
+    if (varlen) return 8192;
+    const long long N = P.N, items_per_seg = 2 * P.count();
     const int sms = 148;
-    if (N <= 1024) return (int)std::max<long long>(128, (N + 127) / 128 * 128);
+    const long long whole = std::max<long long>(128, (N + 127) / 128 * 128);
     double best = 1e300;
-    int best_seg = 2048;
-    for (int seg = 1024; seg <= 8192; seg *= 2) {
-        const long long nseg = (N + seg - 1) / seg;
-        const long long items = chains * nseg;
+    long long best_seg = whole;
+    for (long long seg = 1024;; seg *= 2) {
+        const long long s = std::min(seg, whole);
+        const long long nseg = (N + s - 1) / s;
+        const long long items = items_per_seg * nseg;
         const double rounds = (double)((items + sms - 1) / sms);
-        const double blocks = seg / 128.0;
-        const double per_item = blocks * (nseg > 1 ? 1.25 : 1.0) + 3.0;
+        const double per_item = (s / 128.0) * (nseg > 1 ? 1.4 : 1.0) + 2.0;
         const double cost = rounds * per_item;
         if (cost < best * 0.999) {
             best = cost;
-            best_seg = seg;
+            best_seg = s;
         }
+        if (s == whole) break;
     }
-    return best_seg;
+    return (int)std::min<long long>(best_seg, 1 << 30);
 }
 
 struct WsLayout {
@@ -1417,9 +1228,9 @@ static WsLayout layout(const Problems& P, int seg, bool varlen)
     else
         w.max_items = w.nchains * ((P.N + seg - 1) / seg);
     w.flags = sizeof(WsHeader);
-    w.items = align_up(w.flags + sizeof(int) * (size_t)w.nchains, 256);
+    w.items = align_up(w.flags + sizeof(int) * 2 * (size_t)w.nchains, 256);
     w.incl = align_up(w.items + (varlen ? sizeof(int4) * (size_t)w.max_items : 0), 256);
-    w.end = align_up(w.incl + sizeof(float) * (size_t)w.nchains * 2 * D * D, 256);
+    w.end = align_up(w.incl + sizeof(float) * (size_t)w.nchains * 2 * 2 * D * DV, 256);
     return w;
 }
 
@@ -1451,7 +1262,7 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
         return cudaSuccess;
     }
     if (varlen && P.total == 0 && P.num_seqs == 0) return cudaSuccess;
-    // Clear the header and per-chain counters.
+    // Clear the header and the per-chain counters.
     err = cudaMemsetAsync(ws, 0, w.items, stream);
     if (err != cudaSuccess) return err;
 
@@ -1491,7 +1302,7 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         if (P.total == 0) return cudaSuccess;
     }
-    const long long max_items = w.max_items;
+    const long long max_items = 2 * w.max_items;
     const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(1, max_items));
     auto launch = [&](auto kern) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
