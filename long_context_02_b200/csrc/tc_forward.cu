@@ -73,9 +73,9 @@ constexpr int DV = 64;                           // value columns per work item
 constexpr int C = 128;                           // tokens per block
 constexpr int NUM_THREADS = 512;                 // 4 warpgroups
 // Register split (setmaxnreg, which ptxas also uses to allocate each role):
-// launched at 65536 / 512 = 128 per thread. 128 * (96 + 120 + 120 + 168) =
+// launched at 65536 / 512 = 128 per thread. 128 * (104 + 120 + 128 + 152) =
 // 64512 <= 65536.
-constexpr int REGS_CTRL = 96, REGS_P = 120, REGS_VO = 120, REGS_S = 168;
+constexpr int REGS_CTRL = 104, REGS_P = 120, REGS_VO = 128, REGS_S = 152;
 constexpr uint32_t BOX_BYTES = 128 * 64 * 2;     // one TMA box: 128 rows x 64 bf16
 constexpr uint32_t TILE_BYTES = 2 * BOX_BYTES;   // 128 x 128 bf16
 // Tile region (1024-aligned).
@@ -206,11 +206,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity)
 // Bounded wait. Gives up (returning false) when another role aborted, or
 // after `limit` ns, in which case it records the timeout and raises the
 // CTA-wide abort flag.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort,
-                                          WsHeader* hdr,
-                                          unsigned long long limit = WAIT_LIMIT_NS)
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t* b, uint32_t parity, volatile int* abort,
+                                            WsHeader* hdr, unsigned long long limit)
 {
-    if (mbar_try_wait(b, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(b, parity)) return true;
@@ -223,6 +221,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
             }
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort,
+                                          WsHeader* hdr,
+                                          unsigned long long limit = WAIT_LIMIT_NS)
+{
+    if (mbar_try_wait(b, parity)) return true;
+    return mbar_wait_slow(b, parity, abort, hdr, limit);
 }
 
 // Warp-uniform bounded wait: every lane polls, and the warp proceeds only if
@@ -245,6 +251,16 @@ __device__ __forceinline__ bool group_sync(uint64_t* b, uint32_t& n, volatile in
 __device__ __forceinline__ void fence_proxy_async()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// One lane of a converged warp (the lowest active lane: lane 0 here).
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
 }
 
 __device__ __forceinline__ uint64_t l2_policy_evict_first()
@@ -360,6 +376,50 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
     lo = pack_bf16x2(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
 }
 
+// Pairs of fp32 in one 64-bit register for the packed f32x2 instructions.
+__device__ __forceinline__ uint64_t f2(float a, float b)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2u(uint32_t a, uint32_t b)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ float f2x(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2y(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// bf16x2 word -> fp32 pair (exact).
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) { return f2u(w << 16, w & 0xffff0000u); }
+
+// Pair x -> (hi, lo) bf16x2 words with x = hi + lo to about 2^-16 relative.
+__device__ __forceinline__ void split_pair(uint64_t x, uint32_t& hi, uint32_t& lo)
+{
+    hi = pack_bf16x2(f2x(x), f2y(x));
+    const uint64_t d = sub2(x, bf2_to_f2(hi));
+    lo = pack_bf16x2(f2x(d), f2y(d));
+}
+
 // Shared-memory matrix descriptor: 128-byte swizzle, sm_100 version bit.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
 {
@@ -418,22 +478,6 @@ __device__ __forceinline__ void st_cg_ordered(float* p, float4 w)
     asm volatile("st.global.cg.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(w.x), "f"(w.y),
                  "f"(w.z), "f"(w.w)
                  : "memory");
-}
-
-// Write 64 fp32 values as hi and lo bf16 rows r of two swizzled 128 x 64 boxes.
-__device__ __forceinline__ void store_split_row(uint8_t* hi_box, uint8_t* lo_box, int r,
-                                                const float (&x)[DV])
-{
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint4 h, l;
-        split2(x[8 * c + 0], x[8 * c + 1], h.x, l.x);
-        split2(x[8 * c + 2], x[8 * c + 3], h.y, l.y);
-        split2(x[8 * c + 4], x[8 * c + 5], h.z, l.z);
-        split2(x[8 * c + 6], x[8 * c + 7], h.w, l.w);
-        *reinterpret_cast<uint4*>(hi_box + swz(r, c)) = h;
-        *reinterpret_cast<uint4*>(lo_box + swz(r, c)) = l;
-    }
 }
 
 // ------------------------------------------------------------------ work items
@@ -513,8 +557,9 @@ __device__ __forceinline__ bool next_item(const Params& p, const Smem& sm, uint3
     return it.valid != 0;
 }
 
+// Producer warp: TMA loads (one elected lane issues; the warp waits together).
 __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                              const CUtensorMap* tv, const Smem& sm)
+                              const CUtensorMap* tv, const Smem& sm, int lane)
 {
     uint64_t* bars = sm.bars;
     const int num_items = 2 * (p.cu_seqlens ? *reinterpret_cast<volatile int*>(&p.hdr->num_items)
@@ -528,11 +573,16 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
         const int slot = k & 1;
-        if (!mbar_wait(&bars[B_ITEM_EMPTY0 + slot], ((k >> 1) & 1) ^ 1, sm.abort, p.hdr)) break;
-        const int t = atomicAdd(&p.hdr->ticket, 1);
+        if (!wait_warp(&bars[B_ITEM_EMPTY0 + slot], ((k >> 1) & 1) ^ 1, sm.abort, p.hdr)) break;
+        int t = 0;
+        if (lane == 0) t = atomicAdd(&p.hdr->ticket, 1);
+        t = __shfl_sync(0xffffffffu, t, 0);
         const Item it = make_item(p, t, num_items);
-        sm.ring[slot] = it;
-        mbar_arrive(&bars[B_ITEM_FULL0 + slot]);
+        if (lane == 0) {
+            sm.ring[slot] = it;
+            mbar_arrive(&bars[B_ITEM_FULL0 + slot]);
+        }
+        __syncwarp();
         if (!it.valid) break;
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
@@ -541,25 +591,34 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int y = it.y0 + block_t0(it.len, kb, p.reverse);
                 const int s = nk & 1;
-                ok = mbar_wait(&bars[B_KE0 + s], ((nk >> 1) & 1) ^ 1, sm.abort, p.hdr);
+                ok = wait_warp(&bars[B_KE0 + s], ((nk >> 1) & 1) ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
-                mbar_expect_tx(&bars[B_KF0 + s], TILE_BYTES);
-                tma_load_3d(sm.k(s), tk, &bars[B_KF0 + s], 0, y, it.z, kpol);
-                tma_load_3d(sm.k(s) + BOX_BYTES, tk, &bars[B_KF0 + s], 64, y, it.z, kpol);
+                if (elect_one()) {
+                    mbar_expect_tx(&bars[B_KF0 + s], TILE_BYTES);
+                    tma_load_3d(sm.k(s), tk, &bars[B_KF0 + s], 0, y, it.z, kpol);
+                    tma_load_3d(sm.k(s) + BOX_BYTES, tk, &bars[B_KF0 + s], 64, y, it.z, kpol);
+                }
+                __syncwarp();
                 ++nk;
                 if (pass == 1) {
                     const int sq = nq & 1;
-                    ok = mbar_wait(&bars[B_QE0 + sq], ((nq >> 1) & 1) ^ 1, sm.abort, p.hdr);
+                    ok = wait_warp(&bars[B_QE0 + sq], ((nq >> 1) & 1) ^ 1, sm.abort, p.hdr);
                     if (!ok) break;
-                    mbar_expect_tx(&bars[B_QF0 + sq], TILE_BYTES);
-                    tma_load_3d(sm.q(sq), tq, &bars[B_QF0 + sq], 0, y, it.z, normal);
-                    tma_load_3d(sm.q(sq) + BOX_BYTES, tq, &bars[B_QF0 + sq], 64, y, it.z, normal);
+                    if (elect_one()) {
+                        mbar_expect_tx(&bars[B_QF0 + sq], TILE_BYTES);
+                        tma_load_3d(sm.q(sq), tq, &bars[B_QF0 + sq], 0, y, it.z, normal);
+                        tma_load_3d(sm.q(sq) + BOX_BYTES, tq, &bars[B_QF0 + sq], 64, y, it.z, normal);
+                    }
+                    __syncwarp();
                     ++nq;
                 }
-                ok = mbar_wait(&bars[B_VE0 + s], ((nv >> 1) & 1) ^ 1, sm.abort, p.hdr);
+                ok = wait_warp(&bars[B_VE0 + s], ((nv >> 1) & 1) ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
-                mbar_expect_tx(&bars[B_VF0 + s], BOX_BYTES);
-                tma_load_3d(sm.v(s), tv, &bars[B_VF0 + s], DV * it.half, y, it.z, vpol);
+                if (elect_one()) {
+                    mbar_expect_tx(&bars[B_VF0 + s], BOX_BYTES);
+                    tma_load_3d(sm.v(s), tv, &bars[B_VF0 + s], DV * it.half, y, it.z, vpol);
+                }
+                __syncwarp();
                 ++nv;
             }
         }
@@ -577,41 +636,72 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
     }
 }
 
-__device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
+// K-step offsets of shared-memory descriptors, in the descriptor's 16-byte
+// address units: K-major tiles (two 64-column boxes, 32 bytes per k-step
+// inside a box) and MN-major tiles (16 rows of 128 bytes per k-step).
+__device__ __forceinline__ uint64_t koff_k(int ks)
+{
+    return (uint64_t)((ks >> 2) * (BOX_BYTES >> 4) + (ks & 3) * 2);
+}
+__device__ __forceinline__ uint64_t koff_mn(int ks) { return (uint64_t)(ks * 128); }
+
+// MMA warp: the whole warp waits; one elected lane (lane 0, the warp being
+// converged) issues every MMA and commit, so that each commit tracks all
+// earlier MMAs. Descriptors are built once; each MMA adds a constant k-step
+// offset, which keeps the issue loop short.
+__device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lane)
 {
     uint64_t* bars = sm.bars;
-    const uint32_t vh = smem_u32(sm.vh()), vl = smem_u32(sm.vl());
-    const uint32_t shi = smem_u32(sm.sh()), slo = smem_u32(sm.sl());
+    // Slot s's tile is slot 0's plus a fixed distance, so one base per tensor.
+    const uint64_t dq0 = sdesc(smem_u32(sm.q(0)), 16u, 1024u);
+    const uint64_t dk0 = sdesc(smem_u32(sm.k(0)), 16u, 1024u);
+    const uint64_t dkm0 = sdesc(smem_u32(sm.k(0)), BOX_BYTES, 1024u);
+    const uint64_t dv0 = sdesc(smem_u32(sm.v(0)), 16u, 1024u);
+    const uint64_t dvh = sdesc(smem_u32(sm.vh()), 16u, 1024u);
+    const uint64_t dsh = sdesc(smem_u32(sm.sh()), 16u, 1024u);
+    constexpr uint64_t TILE16 = TILE_BYTES >> 4, BOX16 = BOX_BYTES >> 4;
     // nq, nkv: Q / K-V loads consumed; g: phase-C blocks; n_ds: DS productions;
     // n_vh: decayed-value tiles; n_s: state copies.
     uint32_t nq = 0, nkv = 0, g = 0, n_ds = 0, n_vh = 0, n_s = 0;
+    auto commit = [&](int bar) {
+        if (elect_one()) mma_commit(&bars[bar]);
+        __syncwarp();
+    };
     // DS = K^T Vd (hi and lo) for the K tile in slot sk.
     auto mma4 = [&](int sk, bool accumulate) {
-        const uint32_t kk = smem_u32(sm.k(sk));
+        const uint64_t a = dkm0 + (uint64_t)sk * TILE16;
+        const uint32_t d = tmem + COL_DS;
+        const uint32_t acc0 = accumulate ? 1u : 0u;
+        if (elect_one()) {
 #pragma unroll
-        for (int part = 0; part < 2; ++part)
+            for (int part = 0; part < 2; ++part)
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_ss(tmem + COL_DS, desc_mnmajor(kk, ks), desc_mn64(part ? vl : vh, ks),
-                       IDESC_KV, (accumulate || part || ks) ? 1u : 0u);
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_ss(d, a + koff_mn(ks), dvh + part * BOX16 + koff_mn(ks), IDESC_KV,
+                           (part || ks) ? 1u : acc0);
+        }
+        __syncwarp();
     };
     // SP[g & 1] = Q K^T for phase-C block g (Q slot nq, K slot nkv).
     auto mma1 = [&](uint32_t gg, uint32_t q_use, uint32_t kv_use) -> bool {
         const int sq = q_use & 1, sk = kv_use & 1;
-        if (!mbar_wait(&bars[B_QF0 + sq], (q_use >> 1) & 1, sm.abort, p.hdr)) return false;
-        if (!mbar_wait(&bars[B_KF0 + sk], (kv_use >> 1) & 1, sm.abort, p.hdr)) return false;
+        if (!wait_warp(&bars[B_QF0 + sq], (q_use >> 1) & 1, sm.abort, p.hdr)) return false;
+        if (!wait_warp(&bars[B_KF0 + sk], (kv_use >> 1) & 1, sm.abort, p.hdr)) return false;
         tc_fence_after();
-        const uint32_t qq = smem_u32(sm.q(sq)), kk = smem_u32(sm.k(sk));
+        const uint64_t a = dq0 + (uint64_t)sq * TILE16, b = dk0 + (uint64_t)sk * TILE16;
         const uint32_t d = tmem + COL_SP + 128u * (gg & 1);
+        if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-            mma_ss(d, desc_kmajor(qq, ks), desc_kmajor(kk, ks), IDESC_QK, ks > 0 ? 1u : 0u);
-        mma_commit(&bars[B_SP_FULL0 + (gg & 1)]);
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ss(d, a + koff_k(ks), b + koff_k(ks), IDESC_QK, ks > 0 ? 1u : 0u);
+            mma_commit(&bars[B_SP_FULL0 + (gg & 1)]);
+        }
+        __syncwarp();
         return true;
     };
     Item it;
     for (uint32_t k = 0;; ++k) {
-        if (!next_item(p, sm, k, it, false, 0)) break;
+        if (!next_item(p, sm, k, it, true, lane)) break;
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
@@ -619,20 +709,23 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
             // Phase A: DS accumulates the segment's local state over its blocks.
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int sk = nkv & 1;
-                ok = mbar_wait(&bars[B_KF0 + sk], (nkv >> 1) & 1, sm.abort, p.hdr) &&
-                     mbar_wait(&bars[B_VH_READY], n_vh & 1, sm.abort, p.hdr) &&
-                     (kb > 0 || mbar_wait(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr));
+                ok = wait_warp(&bars[B_KF0 + sk], (nkv >> 1) & 1, sm.abort, p.hdr) &&
+                     wait_warp(&bars[B_VH_READY], n_vh & 1, sm.abort, p.hdr) &&
+                     (kb > 0 || wait_warp(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr));
                 if (!ok) break;
                 ++n_vh;
                 tc_fence_after();
                 mma4(sk, kb > 0);
-                mma_commit(&bars[B_VH_FREE]);
-                mma_commit(&bars[B_KE0 + sk]);
-                mma_commit(&bars[B_VE0 + sk]);
+                if (elect_one()) {
+                    mma_commit(&bars[B_VH_FREE]);
+                    mma_commit(&bars[B_KE0 + sk]);
+                    mma_commit(&bars[B_VE0 + sk]);
+                }
+                __syncwarp();
                 ++nkv;
             }
             if (!ok) break;
-            mma_commit(&bars[B_DS_FULL]);
+            commit(B_DS_FULL);
             ++n_ds;
         }
         // Phase C.
@@ -643,55 +736,64 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
             const int sq = (q0 + kb) & 1, skv = (kv0 + kb) & 1;
             // MMA4: this block's DS, once E_V has decayed its values and E_S
             // has read the previous DS.
-            ok = mbar_wait(&bars[B_VH_READY], n_vh & 1, sm.abort, p.hdr) &&
-                 mbar_wait(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr);
+            ok = wait_warp(&bars[B_VH_READY], n_vh & 1, sm.abort, p.hdr) &&
+                 wait_warp(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr);
             if (!ok) break;
             ++n_vh;
             tc_fence_after();
             mma4(skv, false);
-            mma_commit(&bars[B_DS_FULL]);
-            mma_commit(&bars[B_VH_FREE]);
-            mma_commit(&bars[B_KE0 + skv]);
+            if (elect_one()) {
+                mma_commit(&bars[B_DS_FULL]);
+                mma_commit(&bars[B_VH_FREE]);
+                mma_commit(&bars[B_KE0 + skv]);
+            }
+            __syncwarp();
             ++n_ds;
             // MMA3: OE[g & 1] = Q S_in (hi and lo), once E_S has written the copy.
-            ok = mbar_wait(&bars[B_S_READY], n_s & 1, sm.abort, p.hdr);
+            ok = wait_warp(&bars[B_S_READY], n_s & 1, sm.abort, p.hdr);
             if (!ok) break;
             ++n_s;
             tc_fence_after();
             {
-                const uint32_t qq = smem_u32(sm.q(sq));
+                const uint64_t a = dq0 + (uint64_t)sq * TILE16;
                 const uint32_t d = tmem + COL_OE + (uint32_t)DV * (gg & 1);
+                if (elect_one()) {
 #pragma unroll
-                for (int part = 0; part < 2; ++part)
+                    for (int part = 0; part < 2; ++part)
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_ss(d, desc_kmajor(qq, ks), desc_mn64(part ? slo : shi, ks),
-                               IDESC_QS, (part || ks) ? 1u : 0u);
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_ss(d, a + koff_k(ks), dsh + part * BOX16 + koff_mn(ks), IDESC_QS,
+                                   (part || ks) ? 1u : 0u);
+                    mma_commit(&bars[B_S_FREE]);
+                    mma_commit(&bars[B_QE0 + sq]);
+                }
+                __syncwarp();
             }
-            mma_commit(&bars[B_S_FREE]);
-            mma_commit(&bars[B_QE0 + sq]);
             // MMA1 of the next block, so that E_P overlaps this block's MMA2.
             if (kb + 1 < nb && !(ok = mma1(gg + 1, q0 + kb + 1, kv0 + kb + 1))) break;
             // MMA2: OI = P V (P hi and lo from TMEM), once E_P is done and
             // E_O has read the previous OI.
-            ok = mbar_wait(&bars[B_P_READY0 + (gg & 1)], (gg >> 1) & 1, sm.abort, p.hdr) &&
-                 mbar_wait(&bars[B_O_EMPTY], (gg & 1) ^ 1, sm.abort, p.hdr);
+            ok = wait_warp(&bars[B_P_READY0 + (gg & 1)], (gg >> 1) & 1, sm.abort, p.hdr) &&
+                 wait_warp(&bars[B_O_EMPTY], (gg & 1) ^ 1, sm.abort, p.hdr);
             if (!ok) break;
             tc_fence_after();
             {
-                const uint32_t vv = smem_u32(sm.v(skv));
+                const uint64_t b = dv0 + (uint64_t)skv * BOX16;
                 const uint32_t a = tmem + COL_SP + 128u * (gg & 1);
                 // K-step ks (tokens 16ks..16ks+15) sits in chunk ks/2: hi words
                 // at column 32(ks/2) + 8(ks%2), lo words 16 columns further.
+                if (elect_one()) {
 #pragma unroll
-                for (int part = 0; part < 2; ++part)
+                    for (int part = 0; part < 2; ++part)
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_ts(tmem + COL_OI, a + 32u * (ks >> 1) + 8u * (ks & 1) + 16u * part,
-                               desc_mn64(vv, ks), IDESC_PV, (part || ks) ? 1u : 0u);
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_ts(tmem + COL_OI, a + 32u * (ks >> 1) + 8u * (ks & 1) + 16u * part,
+                                   b + koff_mn(ks), IDESC_PV, (part || ks) ? 1u : 0u);
+                    mma_commit(&bars[B_O_FULL]);
+                    mma_commit(&bars[B_VE0 + skv]);
+                }
+                __syncwarp();
             }
-            mma_commit(&bars[B_O_FULL]);
-            mma_commit(&bars[B_VE0 + skv]);
         }
         if (!ok) break;
         nq += nb;
@@ -699,12 +801,20 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem)
         g += nb;
     }
     // Make sure no MMA is in flight before TMEM is released.
-    mma_commit(&bars[B_FIN]);
+    commit(B_FIN);
     volatile int never = 0;
     mbar_wait(&bars[B_FIN], 0, &never, p.hdr, DRAIN_LIMIT_NS);
+    __syncwarp();
 }
 
 // P group: E_P for every phase-C block.
+//
+// Full blocks take a fast path: in chunks that lie entirely on the causal
+// side of the diagonal, the decay lam^m of consecutive columns is formed by
+// repeated multiplication by lam^2 along two chains (pairs of columns, f32x2),
+// starting from the exact table values, and always toward larger exponents,
+// so underflow only ever reaches values that are zero in fp32 anyway. The
+// diagonal chunk and partial blocks read the exact table per element.
 template <int REV>
 __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
@@ -722,6 +832,8 @@ __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         pw[row] = expf(-slope * (float)row);
         if (row == 0) pw[C] = expf(-slope * (float)C);
         if (!group_sync(&bars[B_P_SYNC], n_sync, sm.abort, p.hdr)) break;
+        const float lam2 = pw[2];
+        const uint64_t L2 = f2(lam2, lam2);
         const int nb = num_blocks(it.len);
         bool ok = true;
         for (int kb = 0; kb < nb && ok; ++kb, ++g) {
@@ -734,34 +846,59 @@ __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
             // Chunk c covers columns 32c..32c+31; warp w holds rows 32w..32w+31,
             // so chunks before (forward) / after (reverse) the diagonal chunk
             // are fully causal and the rest fully masked.
+            const bool full = L == C;
             const bool row_live = REV ? true : row < L;
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t hi[16], lo[16];
                 const bool active = REV ? (c >= w) : (c <= w);
                 if (active) {
                     uint32_t r32[32];
                     tmem_ld32(base + 32 * c, r32);
+                    uint64_t W[16];  // decay of columns (32c + 2e, 32c + 2e + 1)
+                    if (full && c != w) {
+                        // Exponent of column 32c + t: E - t (forward) or E + t (reverse).
+                        const int E = REV ? 32 * c - row : row - 32 * c;
+                        uint64_t wa, wb;  // chains over pairs 15..8 and 7..0 (forward) / 0..7 and 8..15
+                        if (REV) {
+                            wa = f2(pw[E], pw[E + 1]);
+                            wb = f2(pw[E + 16], pw[E + 17]);
+                        } else {
+                            wa = f2(pw[E - 30], pw[E - 31]);
+                            wb = f2(pw[E - 14], pw[E - 15]);
+                        }
+#pragma unroll
+                        for (int step = 0; step < 8; ++step) {
+                            W[REV ? step : 15 - step] = wa;
+                            W[REV ? 8 + step : 7 - step] = wb;
+                            wa = mul2(wa, L2);
+                            wb = mul2(wb, L2);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            float x2[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int j = 32 * c + 2 * e + u;
+                                bool keep;
+                                int m;
+                                if (REV) {
+                                    keep = (c > w || j >= row) && j < L;
+                                    m = j - row;
+                                } else {
+                                    keep = (c < w || j <= row) && row_live;
+                                    m = row - j;
+                                }
+                                x2[u] = keep ? pw[keep ? m : 0] : 0.f;
+                            }
+                            W[e] = f2(x2[0], x2[1]);
+                        }
+                    }
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float x2[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int j = 32 * c + 2 * e + u;
-                            bool keep;
-                            int m;
-                            if (REV) {
-                                keep = (c > w || j >= row) && j < L;
-                                m = j - row;
-                            } else {
-                                keep = (c < w || j <= row) && row_live;
-                                m = row - j;
-                            }
-                            x2[u] = keep ? __uint_as_float(r32[2 * e + u]) * pw[keep ? m : 0] : 0.f;
-                        }
-                        split2(x2[0], x2[1], hi[e], lo[e]);
-                    }
+                    for (int e = 0; e < 16; ++e)
+                        split_pair(mul2(f2u(r32[2 * e], r32[2 * e + 1]), W[e]), hi[e], lo[e]);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
@@ -795,17 +932,19 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         if (!wait_warp(&bars[B_VF0 + s], (nkv >> 1) & 1, sm.abort, p.hdr)) return false;
         if (!wait_warp(&bars[B_VH_FREE], (n_vh & 1) ^ 1, sm.abort, p.hdr)) return false;
         const float f = row < L ? expf(-slope * (float)m) : 0.f;
+        const uint64_t ff = f2(f, f);
         const uint8_t* src = sm.v(s);
-        float x[DV];
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < 8; ++c) {
             const uint4 u = *reinterpret_cast<const uint4*>(src + swz(row, c));
-            x[8 * c + 0] = bf16_lo(u.x) * f; x[8 * c + 1] = bf16_hi(u.x) * f;
-            x[8 * c + 2] = bf16_lo(u.y) * f; x[8 * c + 3] = bf16_hi(u.y) * f;
-            x[8 * c + 4] = bf16_lo(u.z) * f; x[8 * c + 5] = bf16_hi(u.z) * f;
-            x[8 * c + 6] = bf16_lo(u.w) * f; x[8 * c + 7] = bf16_hi(u.w) * f;
+            uint4 h, l;
+            split_pair(mul2(bf2_to_f2(u.x), ff), h.x, l.x);
+            split_pair(mul2(bf2_to_f2(u.y), ff), h.y, l.y);
+            split_pair(mul2(bf2_to_f2(u.z), ff), h.z, l.z);
+            split_pair(mul2(bf2_to_f2(u.w), ff), h.w, l.w);
+            *reinterpret_cast<uint4*>(sm.vh() + swz(row, c)) = h;
+            *reinterpret_cast<uint4*>(sm.vl() + swz(row, c)) = l;
         }
-        store_split_row(sm.vh(), sm.vl(), row, x);
         fence_proxy_async();
         mbar_arrive(&bars[B_VH_READY]);
         ++nkv;
@@ -840,33 +979,35 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
             const int t0 = block_t0(it.len, kb, REV);
             const int L = min(C, it.len - t0);
             const float rowc = expf(-slope * (float)(REV ? max(L - row, 0) : row + 1));
+            const uint64_t rc2 = f2(rowc, rowc);
             const bool store = row < L;
             const long long orow = it.out_row0 + t0 + row;
-#pragma unroll
+#pragma unroll 1
             for (int h = 0; h < 2; ++h) {
                 uint32_t ri[32], re[32];
                 tmem_ld32(lane_addr + COL_OI + 32 * h, ri);
                 tmem_ld32(lane_addr + COL_OE + (uint32_t)DV * (g & 1) + 32 * h, re);
                 tmem_wait_ld();
-                float ov[32];
+                uint64_t ov[16];
 #pragma unroll
-                for (int x = 0; x < 32; ++x)
-                    ov[x] = fmaf(rowc, __uint_as_float(re[x]), __uint_as_float(ri[x]));
+                for (int x = 0; x < 16; ++x)
+                    ov[x] = fma2(rc2, f2u(re[2 * x], re[2 * x + 1]), f2u(ri[2 * x], ri[2 * x + 1]));
                 if (store) {
                     const size_t off = (size_t)orow * D + DV * it.half + 32 * h;
                     if (OUT_F32) {
                         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + off);
 #pragma unroll
                         for (int x = 0; x < 8; ++x)
-                            dst[x] = make_float4(ov[4 * x], ov[4 * x + 1], ov[4 * x + 2], ov[4 * x + 3]);
+                            dst[x] = make_float4(f2x(ov[2 * x]), f2y(ov[2 * x]), f2x(ov[2 * x + 1]),
+                                                 f2y(ov[2 * x + 1]));
                     } else {
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
 #pragma unroll
                         for (int x = 0; x < 4; ++x)
-                            dst[x] = make_uint4(pack_bf16x2(ov[8 * x + 0], ov[8 * x + 1]),
-                                                pack_bf16x2(ov[8 * x + 2], ov[8 * x + 3]),
-                                                pack_bf16x2(ov[8 * x + 4], ov[8 * x + 5]),
-                                                pack_bf16x2(ov[8 * x + 6], ov[8 * x + 7]));
+                            dst[x] = make_uint4(pack_bf16x2(f2x(ov[4 * x + 0]), f2y(ov[4 * x + 0])),
+                                                pack_bf16x2(f2x(ov[4 * x + 1]), f2y(ov[4 * x + 1])),
+                                                pack_bf16x2(f2x(ov[4 * x + 2]), f2y(ov[4 * x + 2])),
+                                                pack_bf16x2(f2x(ov[4 * x + 3]), f2y(ov[4 * x + 3])));
                     }
                 }
             }
@@ -878,7 +1019,8 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
 }
 
 // S group: E_S (the fp32 state, row a of this item's 128 x 64 state per
-// thread), the hi/lo state copies for MMA3, and the scan between segments.
+// thread, kept as 32 f32x2 pairs), the hi/lo state copies for MMA3, and the
+// scan between segments.
 template <int REV>
 __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
@@ -886,31 +1028,42 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
     const int a = ((warp & 3) << 5) | lane;  // TMEM lane = key dim a
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) << 5) << 16);
     uint32_t n_ds = 0, n_s = 0, n_sync = 0;
-    float S[DV];
+    uint64_t S[DV / 2];
     Item it;
-    // DS row a -> x (with S = dL * S + DS when accumulate).
+    // DS row a -> S (S = dL * S + DS when accumulate).
     auto read_ds = [&](float dL, bool accumulate) -> bool {
         if (!wait_warp(&bars[B_DS_FULL], n_ds & 1, sm.abort, p.hdr)) return false;
         tc_fence_after();
+        const uint64_t d2 = f2(dL, dL);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             uint32_t r[32];
             tmem_ld32(lane_addr + COL_DS + 32 * h, r);
             tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 32; ++x)
-                S[32 * h + x] = accumulate ? fmaf(dL, S[32 * h + x], __uint_as_float(r[x]))
-                                           : __uint_as_float(r[x]);
+            for (int x = 0; x < 16; ++x) {
+                const uint64_t ds = f2u(r[2 * x], r[2 * x + 1]);
+                S[16 * h + x] = accumulate ? fma2(d2, S[16 * h + x], ds) : ds;
+            }
         }
         tc_fence_before();
         mbar_arrive(&bars[B_DS_EMPTY]);
         ++n_ds;
         return true;
     };
-    // Hi/lo copies of the state for the next MMA3.
+    // Hi/lo copies of the state (row a of two swizzled 128 x 64 boxes) for the next MMA3.
     auto publish_copy = [&]() -> bool {
         if (!wait_warp(&bars[B_S_FREE], (n_s & 1) ^ 1, sm.abort, p.hdr)) return false;
-        store_split_row(sm.sh(), sm.sl(), a, S);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint4 h, l;
+            split_pair(S[4 * c + 0], h.x, l.x);
+            split_pair(S[4 * c + 1], h.y, l.y);
+            split_pair(S[4 * c + 2], h.z, l.z);
+            split_pair(S[4 * c + 3], h.w, l.w);
+            *reinterpret_cast<uint4*>(sm.sh() + swz(a, c)) = h;
+            *reinterpret_cast<uint4*>(sm.sl() + swz(a, c)) = l;
+        }
         fence_proxy_async();
         mbar_arrive(&bars[B_S_READY]);
         ++n_s;
@@ -927,7 +1080,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
             if (!read_ds(0.f, false)) break;  // S = S_loc
         } else {
 #pragma unroll
-            for (int x = 0; x < DV; ++x) S[x] = 0.f;
+            for (int x = 0; x < DV / 2; ++x) S[x] = 0ull;
         }
         // Incoming state: the predecessor's inclusive prefix (zero for the first segment).
         const float* src = p.incl + (((size_t)chain2 * 2 + ((it.p_ord - 1) & 1)) * D + a) * DV;
@@ -955,19 +1108,19 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
             // S_prev = the predecessor's prefix; with a successor, publish
             // lam^len S_prev + S_loc. Phase C continues from S_prev.
             const float dl = expf(-slope * (float)it.len);
+            const uint64_t dl2 = f2(dl, dl);
             float* dst = p.incl + (((size_t)chain2 * 2 + (it.p_ord & 1)) * D + a) * DV;
             const bool has_prev = it.p_ord > 0;
 #pragma unroll
             for (int x = 0; x < DV / 4; ++x) {
                 const float4 w = has_prev ? ld_cg_ordered(src + 4 * x) : make_float4(0.f, 0.f, 0.f, 0.f);
-                if (has_succ)
-                    st_cg_ordered(dst + 4 * x,
-                                  make_float4(fmaf(dl, w.x, S[4 * x + 0]), fmaf(dl, w.y, S[4 * x + 1]),
-                                              fmaf(dl, w.z, S[4 * x + 2]), fmaf(dl, w.w, S[4 * x + 3])));
-                S[4 * x + 0] = w.x;
-                S[4 * x + 1] = w.y;
-                S[4 * x + 2] = w.z;
-                S[4 * x + 3] = w.w;
+                const uint64_t w0 = f2(w.x, w.y), w1 = f2(w.z, w.w);
+                if (has_succ) {
+                    const uint64_t o0 = fma2(dl2, w0, S[2 * x]), o1 = fma2(dl2, w1, S[2 * x + 1]);
+                    st_cg_ordered(dst + 4 * x, make_float4(f2x(o0), f2y(o0), f2x(o1), f2y(o1)));
+                }
+                S[2 * x] = w0;
+                S[2 * x + 1] = w1;
             }
         }
         if (has_succ) {
@@ -990,7 +1143,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
                                                     DV * it.half);
 #pragma unroll
             for (int x = 0; x < DV / 4; ++x)
-                dst[x] = make_float4(S[4 * x], S[4 * x + 1], S[4 * x + 2], S[4 * x + 3]);
+                dst[x] = make_float4(f2x(S[2 * x]), f2y(S[2 * x]), f2x(S[2 * x + 1]), f2y(S[2 * x + 1]));
         }
     }
 }
@@ -1054,8 +1207,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_CTRL));
-        if (warp == 0 && lane == 0) producer_role(p, &tq, &tk, &tv, sm);
-        if (warp == 1 && lane == 0) mma_role(p, sm, tmem);
+        if (warp == 0) producer_role(p, &tq, &tk, &tv, sm, lane);
+        if (warp == 1) mma_role(p, sm, tmem, lane);
     } else if (warp < 8) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_P));
         p_role<REV>(p, sm, tmem, warp, lane);
