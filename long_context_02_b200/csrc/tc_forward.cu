@@ -1255,6 +1255,35 @@ __global__ void __launch_bounds__(1024) plan_varlen_kernel(const int* cu, int nu
     }
     __syncthreads();
     const int maxseg = s_max;
+    if (maxseg == 1 && num_seqs <= 8192) {
+        // One segment per sequence: no item waits on another, so order the
+        // sequences longest first (ties by index) to shorten the tail.
+        auto len_of = [&](int s) -> long long { return (long long)cu[s + 1] - cu[s]; };
+        __shared__ int s_count;
+        if (tid == 0) s_count = 0;
+        __syncthreads();
+        for (int s = tid; s < num_seqs; s += blockDim.x) {
+            const long long Ls = len_of(s);
+            if (Ls <= 0) continue;
+            atomicAdd(&s_count, 1);
+            int rank = 0;
+            for (int s2 = 0; s2 < num_seqs; ++s2) {
+                const long long L2 = len_of(s2);
+                rank += (L2 > Ls || (L2 == Ls && s2 < s)) ? 1 : 0;
+            }
+            for (int h = 0; h < H; ++h) {
+                const long long t = (long long)rank * H + h;
+                if (t < max_items) items[t] = make_int4(s * H + h, 0, 1, 0);
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const long long n = (long long)s_count * H;
+            hdr->num_items = (int)min(n, (long long)max_items);
+            if (n > max_items) atomicExch(&hdr->status, (int)LA_ERR_INVALID_ARG);
+        }
+        return;
+    }
     long long offset = 0;
     for (int pp = 0; pp < maxseg; ++pp) {
         int running = 0;
@@ -1345,7 +1374,13 @@ static int num_sms()
 static int choose_seg(const Problems& P, int seg_tuning, bool varlen)
 {
     if (seg_tuning > 0) return seg_tuning;
-    if (varlen) return 8192;
+    if (varlen) {
+        // With enough (sequence, head, half) items to keep every SM busy, each
+        // sequence is one segment (no scan; the planner orders them longest
+        // first); otherwise segments of 8K tokens add the parallelism.
+        const long long pairs = 2LL * P.num_seqs * P.H;
+        return pairs >= 4LL * 148 ? (1 << 30) : 8192;
+    }
     const long long N = P.N, items_per_seg = 2 * P.count();
     const int sms = 148;
     const long long whole = std::max<long long>(128, (N + 127) / 128 * 128);
