@@ -249,30 +249,50 @@ def run_ours(args):
                 "kernel": "tc_forward_kernel", "algorithmic_bytes": Bytes}
 
     # End to end through the C ABI with host buffers: H2D of Q,K,V from pinned
-    # memory, the call, D2H of O and the state, all inside the timed region.
+    # memory, the calls, D2H of O and the state, all inside the timed region.
+    # The heads are processed in groups on three streams (copy in, compute,
+    # copy out), so one group's copies overlap another group's prefill: the
+    # way a caller holding host tensors would drive the library.
     e2e = None
     if not args.no_e2e:
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         hst = torch.empty(st.shape, dtype=st.dtype).pin_memory()
+        groups = 8
+        hg = H_ // groups
+        ws_g = L.workspace(L.LA_OP_PREFILL, B_, hg, N_, D_, 0, torch.bfloat16, dev)
+        s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
 
         def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            L.la_prefill(q, k, v, s, o, st, ws)
-            ho.copy_(o, non_blocking=True)
-            hst.copy_(st, non_blocking=True)
+            cur = torch.cuda.current_stream()
+            s_in.wait_stream(cur)
+            for g in range(groups):
+                h = slice(g * hg, (g + 1) * hg)
+                with torch.cuda.stream(s_in):
+                    for dst, src in ((q, hq), (k, hk), (v, hv)):
+                        dst[:, h].copy_(src[:, h], non_blocking=True)
+                    loaded = s_in.record_event()
+                s_cmp.wait_event(loaded)
+                L.la_prefill(q[:, h], k[:, h], v[:, h], s[h], o[:, h], st[:, h], ws_g, stream=s_cmp)
+                done = s_cmp.record_event()
+                s_out.wait_event(done)
+                with torch.cuda.stream(s_out):
+                    ho[:, h].copy_(o[:, h], non_blocking=True)
+                    hst[:, h].copy_(st[:, h], non_blocking=True)
+            cur.wait_stream(s_out)
 
         for _ in range(2):
             e2e_step()
+        torch.cuda.synchronize()
+        assert L.la_read_device_status(ws_g) == L.LA_OK
         e2e_steps = max(2, min(args.steps, 20))
         ms_e2e = timed(e2e_step, e2e_steps, world)
         h2d = 3 * q.numel() * q.element_size()
         d2h = o.numel() * o.element_size() + st.numel() * 4
         e2e = {"value": round(world * F / (ms_e2e * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                "ms_per_step": round(ms_e2e, 4), "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+               "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "schedule": f"{groups} head groups, copy-in / prefill / copy-out on 3 streams"}
         del hq, hk, hv, ho, hst
 
     secondary = {} if args.no_secondary else run_secondary(args, L, inputs, dev, world, pk)
