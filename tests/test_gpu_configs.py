@@ -94,6 +94,30 @@ def test_long_context_1m():
     assert_close(np.stack([f64(st[0, h]) for h in hs])[None], st_ref, TOL_BF16, "state")
 
 
+def test_few_heads_long_scan():
+    """Few chains, long sequence: the default tuning cuts each chain into many
+    segments, so the chunk-parallel scan carries the state across dozens of
+    segments (and the time-reversed scan does for the backward legs)."""
+    B, H, N, d = 1, 4, 65536, 128
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.bfloat16, DEV, seed=1006)
+    o = torch.empty(q.shape, dtype=torch.float32, device=DEV)
+    st = torch.empty((B, H, d, d), dtype=torch.float32, device=DEV)
+    ws = L.workspace(L.LA_OP_PREFILL, B, H, N, d)
+    L.la_prefill(q, k, v, s, o, st, ws)
+    assert L.la_read_device_status(ws) == L.LA_OK
+    hs = list(range(H))
+    o_ref, st_ref = oracle.recurrence(_heads(q, hs), _heads(k, hs), _heads(v, hs), lam(s))
+    assert_close(_heads(o, hs), o_ref, TOL_BF16, "O")
+    assert_close(f64(st), st_ref, TOL_BF16, "state")
+    do = inputs.grad_output(q.shape, torch.bfloat16, DEV, seed=1007)
+    dq, dk, dv = L.backward(do, q, k, v, s, out_dtype=torch.float32)
+    rq, rk, rv = oracle.backward_recurrence(_heads(do, hs), _heads(q, hs), _heads(k, hs),
+                                            _heads(v, hs), lam(s))
+    assert_close(_heads(dq, hs), rq, TOL_BF16, "dQ")
+    assert_close(_heads(dk, hs), rk, TOL_BF16, "dK")
+    assert_close(_heads(dv, hs), rv, TOL_BF16, "dV")
+
+
 def test_decode_batch_256():
     B, H, d = 256, 64, 128
     q, k, v, state, s = inputs.decode_inputs(B, H, d, torch.bfloat16, DEV, seed=1003)

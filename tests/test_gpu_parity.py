@@ -127,6 +127,28 @@ def test_varlen(seg):
     assert torch.all(st[1] == 0)
 
 
+def test_varlen_many_items_longest_first():
+    """Enough (sequence, head, half) items that each sequence is one segment and
+    the planner orders them by length (empty, one-token, partial and whole
+    blocks among them); heads 0 and 63 checked by the quadratic oracle."""
+    lengths = [0, 300, 1, 128, 0, 1000, 129, 50, 2048, 7]
+    H = 64
+    q, k, v, cu, s = inputs.varlen_inputs(lengths, H, 128, torch.bfloat16, DEV, seed=15)
+    S = len(lengths)
+    o = torch.full(q.shape, float("nan"), dtype=torch.float32, device=DEV)
+    st = torch.full((S, H, 128, 128), float("nan"), dtype=torch.float32, device=DEV)
+    ws = L.workspace(L.LA_OP_PREFILL_VARLEN, 1, H, q.shape[1], 128, S, torch.bfloat16)
+    L.la_prefill_varlen(cu, q, k, v, s, o, st, ws)
+    assert L.la_read_device_status(ws) == L.LA_OK
+    hs = [0, 63]
+    sub = lambda t: np.stack([f64(t[h]) for h in hs])
+    o_ref, st_ref = oracle.forward_varlen(cu.cpu().numpy(), sub(q), sub(k), sub(v), lam(s)[hs])
+    assert_close(sub(o), o_ref, TOL_BF16, "O (heads 0, 63)")
+    assert_close(np.stack([f64(st[:, h]) for h in hs], axis=1), st_ref, TOL_BF16, "states")
+    assert torch.all(st[0] == 0) and torch.all(st[4] == 0)
+    assert not torch.isnan(o).any()
+
+
 def test_varlen_matches_separate_calls():
     lengths = [513, 1200, 64]
     q, k, v, cu, s = inputs.varlen_inputs(lengths, 2, 128, torch.bfloat16, DEV, seed=6)
