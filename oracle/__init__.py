@@ -90,24 +90,31 @@ class Oracle:
         lib = ctypes.CDLL(path or build())
         P, L, I, D = ctypes.c_void_p, ctypes.c_long, ctypes.c_int, ctypes.c_double
         lib.oracle_forward.argtypes = [I, P, P, P, P, P, P, P, P, P, L]
+        lib.oracle_forward_from_state.argtypes = [I, P, P, P, P, P, P, P, P, P, P, L]
         lib.oracle_recurrence.argtypes = [I, P, P, P, P, P, P, P, P, P, P, L, I]
         lib.oracle_backward.argtypes = [I, P, P, P, P, P, P, P, P, P, P, L]
         lib.oracle_decode.argtypes = [P, P, P, P, P, P, L, L]
         lib.oracle_forward_rows.argtypes = [P, P, P, P, L, P, L, D]
-        for f in ("oracle_forward", "oracle_recurrence", "oracle_backward", "oracle_decode",
+        for f in ("oracle_forward", "oracle_forward_from_state", "oracle_recurrence", "oracle_backward", "oracle_decode",
                   "oracle_forward_rows"):
             getattr(lib, f).restype = None
         self.lib = lib
 
-    def forward(self, q, k, v, lam):
-        """Quadratic form over [B,H,N,d]. Returns (O [B,H,N,d], state [B,H,d,d])."""
+    def forward(self, q, k, v, lam, state_in=None):
+        """Quadratic form over [B,H,N,d]. Returns (O [B,H,N,d], state [B,H,d,d]).
+        state_in [B,H,d,d]: the state of a prefix before token 0 (None = no prefix)."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, H, N, d = q.shape
         ro, ln, so, lp = _dense_problems(B, H, N, lam)
         o = _out(q.shape)
         st = _out((B, H, d, d))
-        self.lib.oracle_forward(B * H, _p(ro), _p(ln), _p(so), _p(lp), _p(q), _p(k), _p(v),
-                                _p(o), _p(st), d)
+        if state_in is None:
+            self.lib.oracle_forward(B * H, _p(ro), _p(ln), _p(so), _p(lp), _p(q), _p(k), _p(v),
+                                    _p(o), _p(st), d)
+        else:
+            si = _f64(state_in).reshape(B, H, d, d)
+            self.lib.oracle_forward_from_state(B * H, _p(ro), _p(ln), _p(so), _p(lp), _p(q),
+                                               _p(k), _p(v), _p(si), _p(o), _p(st), d)
         return o, st
 
     def recurrence(self, q, k, v, lam, state_in=None, reverse=False, want_o=True):
@@ -122,26 +129,33 @@ class Oracle:
                                    _p(o), _p(si), _p(st), d, 1 if reverse else 0)
         return o, st
 
-    def forward_varlen(self, cu_seqlens, q, k, v, lam):
-        """Quadratic form per packed sequence, [H,T,d]. Returns (O, state [S,H,d,d])."""
+    def forward_varlen(self, cu_seqlens, q, k, v, lam, state_in=None):
+        """Quadratic form per packed sequence, [H,T,d]. Returns (O, state [S,H,d,d]).
+        state_in [S,H,d,d]: each sequence's prefix state (None = no prefix)."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         H, T, d = q.shape
         ro, ln, so, lp = _varlen_problems(cu_seqlens, H, T, lam)
         o = _out(q.shape)
         st = _out((len(cu_seqlens) - 1, H, d, d))
-        self.lib.oracle_forward(len(ro), _p(ro), _p(ln), _p(so), _p(lp), _p(q), _p(k), _p(v),
-                                _p(o), _p(st), d)
+        if state_in is None:
+            self.lib.oracle_forward(len(ro), _p(ro), _p(ln), _p(so), _p(lp), _p(q), _p(k),
+                                    _p(v), _p(o), _p(st), d)
+        else:
+            si = _f64(state_in).reshape(len(cu_seqlens) - 1, H, d, d)
+            self.lib.oracle_forward_from_state(len(ro), _p(ro), _p(ln), _p(so), _p(lp), _p(q),
+                                               _p(k), _p(v), _p(si), _p(o), _p(st), d)
         return o, st
 
-    def recurrence_varlen(self, cu_seqlens, q, k, v, lam, want_o=True):
+    def recurrence_varlen(self, cu_seqlens, q, k, v, lam, want_o=True, state_in=None):
         """Token recurrence per packed sequence, [H,T,d]. Returns (O, state [S,H,d,d])."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         H, T, d = q.shape
         ro, ln, so, lp = _varlen_problems(cu_seqlens, H, T, lam)
         o = _out(q.shape) if want_o else None
         st = _out((len(cu_seqlens) - 1, H, d, d))
+        si = None if state_in is None else _f64(state_in)
         self.lib.oracle_recurrence(len(ro), _p(ro), _p(ln), _p(so), _p(lp), _p(q), _p(k),
-                                   _p(v), _p(o), None, _p(st), d, 0)
+                                   _p(v), _p(o), _p(si), _p(st), d, 0)
         return o, st
 
     def forward_rows(self, q, k, v, lam, rows):

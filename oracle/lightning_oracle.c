@@ -77,6 +77,36 @@ void oracle_forward_one(const double* q, const double* k, const double* v,
     free(pw);
 }
 
+/* (1) continued from an incoming state S_in: the state of a prefix of tokens
+ * that come before token 0 (a cached prefix, "MiniMax-01: Scaling Foundation
+ * Models with Lightning Attention | Summary", section 3: inference inputs
+ * whose earlier segments were already computed). Every prefix token j < 0
+ * enters (1) through S_in = sum_{j<0} lam^(-1-j) k_j^T v_j, so
+ *
+ *   O_i   = lam^(i+1) q_i S_in + sum_{0 <= j <= i} lam^(i-j) (q_i . k_j) v_j
+ *   state = lam^N S_in + sum_{0 <= j < N} lam^(N-1-j) k_j^T v_j
+ *
+ * The second terms are (1) over the tokens 0..N-1; the first are added here.
+ * state may be NULL; N may be 0 (then state = S_in). */
+void oracle_forward_from_state_one(const double* q, const double* k, const double* v,
+                                   const double* state_in, double* o, double* state, long N,
+                                   long d, double lam)
+{
+    oracle_forward_one(q, k, v, o, state, N, d, lam);
+    for (long i = 0; i < N; ++i) {
+        double w = pow(lam, (double)(i + 1));
+        for (long b = 0; b < d; ++b) {
+            double s = 0.0;
+            for (long a = 0; a < d; ++a) s += q[i * d + a] * state_in[a * d + b];
+            o[i * d + b] += w * s;
+        }
+    }
+    if (state) {
+        double w = pow(lam, (double)N);
+        for (long a = 0; a < d * d; ++a) state[a] += w * state_in[a];
+    }
+}
+
 /* (1) evaluated only at the given rows of one problem: out[r] = O_{rows[r]}. */
 void oracle_forward_rows(const double* q, const double* k, const double* v,
                          const long* rows, long nrows, double* out, long d, double lam)
@@ -188,6 +218,21 @@ void oracle_forward(int nprob, const long* row_off, const long* len, const long*
             continue;
         }
         oracle_forward_one(q + r, k + r, v + r, o + r, st, len[p], d, lam[p]);
+    }
+}
+
+/* Batched (1) from incoming states: state_in and state share st_off. */
+void oracle_forward_from_state(int nprob, const long* row_off, const long* len, const long* st_off,
+                               const double* lam, const double* q, const double* k,
+                               const double* v, const double* state_in, double* o, double* state,
+                               long d)
+{
+    #pragma omp parallel for schedule(dynamic)
+    for (int p = 0; p < nprob; ++p) {
+        long r = row_off[p] * d;
+        const double* si = state_in + st_off[p] * d * d;
+        double* st = state ? state + st_off[p] * d * d : NULL;
+        oracle_forward_from_state_one(q + r, k + r, v + r, si, o + r, st, len[p], d, lam[p]);
     }
 }
 

@@ -16,6 +16,10 @@ What pins what:
   decode chain == last rows of the prefill   -> decode
   <dO,O> = <dQ,Q> = <dK,K> = <dV,V>           -> backward
   varlen == per-sequence calls               -> forward_varlen, recurrence_varlen
+  exact prefix folded into the state         -> forward / recurrence with state_in
+  cutting a sequence and carrying the state  -> forward / recurrence with state_in
+  all-ones closed form with a constant state -> forward with state_in
+  varlen with states == per-sequence calls   -> forward_varlen with state_in
 """
 from __future__ import annotations
 
@@ -259,6 +263,89 @@ def pin_varlen_is_per_sequence(orc, seed=8):
             np.testing.assert_allclose(st[s], st_s[0], rtol=1e-13, atol=1e-14)
 
 
+def _floats(rows, shape):
+    return np.array([[float(x) for x in r] for r in rows], dtype=np.float64).reshape(shape)
+
+
+def pin_state_in_exact_prefix(orc, seed=9):
+    """A prefix of m tokens folded into S_in (its exact state) and the n tokens
+    after it reproduce the exact rows and final state of the whole sequence
+    (lam = 1/2 and small integers: every value is exact in fp64)."""
+    rng = np.random.default_rng(seed)
+    lam = Fraction(1, 2)
+    for (m, n, d) in ((1, 1, 1), (3, 4, 2), (4, 7, 3), (5, 0, 2), (2, 6, 4)):
+        N = m + n
+        q, k, v = (_rand_int(rng, (N, d)) for _ in range(3))
+        O, S = _frac_forward(_as_frac(q), _as_frac(k), _as_frac(v), lam)
+        _, Sp = _frac_forward(_as_frac(q[:m]), _as_frac(k[:m]), _as_frac(v[:m]), lam)
+        s_in = _floats(Sp, (1, 1, d, d))
+        args = [x[m:].reshape(1, 1, n, d) for x in (q, k, v)]
+        want_o, want_s = _floats(O[m:], (n, d)), _floats(S, (d, d))
+        for fn in (orc.forward, orc.recurrence):
+            o, st = fn(*args, np.array([0.5]), state_in=s_in)
+            assert np.array_equal(o[0, 0], want_o), (fn.__name__, m, n, d, o[0, 0], want_o)
+            assert np.array_equal(st[0, 0], want_s), (fn.__name__, m, n, d, st[0, 0], want_s)
+
+
+def pin_state_in_split_invariance(orc, seed=10):
+    """Cutting a sequence at any m and carrying the state across the cut gives
+    rows m.. and the final state of the uncut sequence."""
+    rng = np.random.default_rng(seed)
+    B, H, N, d = 2, 3, 60, 6
+    q, k, v = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    lam = np.array([0.45, 0.9, 0.999])
+    o_full, s_full = orc.forward(q, k, v, lam)
+    to = 1e-12 * np.abs(o_full).max()
+    ts = 1e-12 * np.abs(s_full).max()
+    for m in (0, 1, 17, 59, 60):
+        _, s_m = orc.forward(q[:, :, :m], k[:, :, :m], v[:, :, :m], lam)
+        tail = [x[:, :, m:] for x in (q, k, v)]
+        for fn in (orc.forward, orc.recurrence):
+            o2, s2 = fn(*tail, lam, state_in=s_m)
+            np.testing.assert_allclose(o2, o_full[:, :, m:], rtol=1e-11, atol=to)
+            np.testing.assert_allclose(s2, s_full, rtol=1e-11, atol=ts)
+
+
+def pin_state_in_all_ones(orc):
+    """q = k = v = 1 and S_in = c in every entry:
+    O_i[b] = lam^(i+1) d c + d (1 - lam^(i+1)) / (1 - lam),
+    state  = lam^N c + (1 - lam^N) / (1 - lam)."""
+    N, d, c = 200, 8, 2.5
+    lam = np.array([0.3, 0.9, 0.999])
+    ones = np.ones((1, 3, N, d))
+    s_in = np.full((1, 3, d, d), c)
+    i = np.arange(N)[None, :, None]
+    l = lam[:, None, None]
+    want_o = (l ** (i + 1) * d * c + d * (1 - l ** (i + 1)) / (1 - l)) * np.ones((3, N, d))
+    want_s = (lam ** N * c + (1 - lam ** N) / (1 - lam))[:, None, None] * np.ones((3, d, d))
+    o, s = orc.forward(ones, ones, ones, lam, state_in=s_in)
+    np.testing.assert_allclose(o[0], want_o, rtol=1e-12)
+    np.testing.assert_allclose(s[0], want_s, rtol=1e-12)
+
+
+def pin_state_in_varlen_is_per_sequence(orc, seed=11):
+    rng = np.random.default_rng(seed)
+    H, d = 2, 4
+    lengths = [5, 0, 1, 9]
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    T = int(cu[-1])
+    q, k, v = (rng.standard_normal((H, T, d)) for _ in range(3))
+    s_in = rng.standard_normal((len(lengths), H, d, d))
+    lam = np.array([0.5, 0.9])
+    for fn, seq_fn in ((orc.forward_varlen, orc.forward),
+                       (orc.recurrence_varlen, orc.recurrence)):
+        o, st = fn(cu, q, k, v, lam, state_in=s_in)
+        for s, L in enumerate(lengths):
+            a, b = cu[s], cu[s + 1]
+            if L == 0:
+                assert np.array_equal(st[s], s_in[s])
+                continue
+            o_s, st_s = seq_fn(q[None, :, a:b], k[None, :, a:b], v[None, :, a:b], lam,
+                               state_in=s_in[s][None])
+            np.testing.assert_allclose(o[:, a:b], o_s[0], rtol=1e-13, atol=1e-14)
+            np.testing.assert_allclose(st[s], st_s[0], rtol=1e-13, atol=1e-14)
+
+
 ALL_PINS = [
     pin_hand_fixture,
     pin_rational_brute_force,
@@ -271,4 +358,8 @@ ALL_PINS = [
     pin_decode_chain,
     pin_backward_identities,
     pin_varlen_is_per_sequence,
+    pin_state_in_exact_prefix,
+    pin_state_in_split_invariance,
+    pin_state_in_all_ones,
+    pin_state_in_varlen_is_per_sequence,
 ]

@@ -53,6 +53,21 @@ MUTANTS = [
     ("backward_dv_swapped_rows",
      "double wv = pw[i - j] * dot(q + i * d, k + j * d, d);",
      "double wv = pw[i - j] * dot(q + j * d, k + i * d, d);"),
+    ("from_state_exponent_off_by_one",
+     "double w = pow(lam, (double)(i + 1));",
+     "double w = pow(lam, (double)i);"),
+    ("from_state_transposed",
+     "s += q[i * d + a] * state_in[a * d + b];",
+     "s += q[i * d + a] * state_in[b * d + a];"),
+    ("from_state_state_decay_off_by_one",
+     "double w = pow(lam, (double)N);",
+     "double w = pow(lam, (double)(N > 0 ? N - 1 : 0));"),
+    ("from_state_drops_state_term",
+     "state[a] += w * state_in[a];",
+     "state[a] += 0.0 * state_in[a];"),
+    ("recurrence_ignores_state_in",
+     "if (state_in) memcpy(S, state_in",
+     "if (0) memcpy(S, state_in"),
     ("varlen_zero_length_state_not_cleared",
      "if (st) for (long a = 0; a < d * d; ++a) st[a] = 0.0;\n            continue;",
      "continue;"),
