@@ -363,6 +363,23 @@ def run_secondary(args, L, inputs, dev, world, pk):
                        "GB/s_algorithmic": round(nbytes / (ms * 1e-3) / 1e9, 1),
                        "flop_convention": "B*H*N*(10d^2 + 10*256*d)"}
     del q, k, v, do, dq, dk, dv, ws
+    # prefill continued from a cached prefix's state (state advanced in place)
+    q, k, v, s = inputs.prefill_inputs(1, 64, 32768, 128, torch.bfloat16, dev, seed=15)
+    st = inputs.state_inputs(1, 64, 128, dev, seed=16)
+    o = torch.empty_like(q)
+    ws = L.workspace(L.LA_OP_PREFILL, 1, 64, 32768, 128, 0, torch.bfloat16, dev)
+    fn = lambda: L.la_prefill_with_state(q, k, v, s, st, o, st, ws)
+    for _ in range(3):
+        fn()
+    ms = timed(fn, steps, world)
+    F = prefill_flops(1, 64, 32768)
+    nbytes = prefill_bytes(1, 64, 32768) + st.numel() * 4
+    out["prefill_with_state"] = {
+        "workload": "prefill from a cached prefix's state B=1 H=64 N=32768 d=128 bf16, "
+                    "state in place",
+        "ms": round(ms, 4), "TFLOP/s": round(world * F / (ms * 1e-3) / 1e12, 2),
+        "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+    del q, k, v, st, o, ws
     if not args.quick:
         # varlen: 16 sequences of U{1024..65536} tokens, packed
         lengths = inputs.varlen_lengths(16, 1024, 65536, seed=0)

@@ -106,6 +106,43 @@ LA_API int la_prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q,
                              size_t ws_bytes, la_stream_t stream);
 
 /*
+ * Prefill continued from an incoming state: the inputs are the tokens that
+ * follow a prefix whose state is already known (a cached prefix, or the
+ * previous piece of a prefill cut into pieces; "MiniMax-01 ... | Summary",
+ * section 3: inference inputs with cached prefixes that reuse the earlier
+ * segments' computation, and section 3.3's batches of cached inputs). With
+ * S_in the state after the prefix, for every (sequence, head):
+ *     O_i   = lam^(i+1) q_i S_in + sum_{j <= i} lam^(i-j) (q_i . k_j) v_j
+ *     state = lam^N S_in + sum_j lam^(N-1-j) k_j^T v_j
+ * so that prefill(prefix) followed by this call on the rest gives the rows
+ * and the final state of one prefill over the whole sequence.
+ *   state_in   in   [B][H][d][d] fp32, not NULL; may be the same array as
+ *                   state_out (the state is then advanced in place); any
+ *                   other overlap with an output is undefined
+ * Every other argument, result and error is as for la_prefill (N may be 0:
+ * state_out then receives state_in).
+ */
+LA_API int la_prefill_with_state(const void* q, const void* k, const void* v,
+                                 const float* slopes, const float* state_in, void* o,
+                                 float* state_out, int B, int H, long long N, int d, int in_t,
+                                 int out_t, void* workspace, size_t ws_bytes, la_stream_t stream);
+
+/*
+ * la_prefill_varlen continued from one incoming state per (sequence, head):
+ *   state_in   in   [num_seqs][H][d][d] fp32, not NULL; may be the same array
+ *                   as state_out
+ * The operator per sequence is that of la_prefill_with_state; a zero-length
+ * sequence's final state is its incoming state. Every other argument, result
+ * and error is as for la_prefill_varlen; the workspace size is that of
+ * LA_OP_PREFILL_VARLEN.
+ */
+LA_API int la_prefill_varlen_with_state(const int* cu_seqlens, int num_seqs, const void* q,
+                                        const void* k, const void* v, const float* slopes,
+                                        const float* state_in, void* o, float* state_out, int H,
+                                        long long total, int d, int in_t, int out_t,
+                                        void* workspace, size_t ws_bytes, la_stream_t stream);
+
+/*
  * One decode step for a batch of B sequences ("MiniMax-01 ... | Summary",
  * section 3.3: the memory-bound single-token step, fused into one kernel):
  *     S <- lam_h S + k^T v     then     o = q S

@@ -25,7 +25,8 @@ LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE, LA_OP_BACKWARD = 0, 1, 2, 3
 
 EXPORTED = ["la_workspace_bytes", "la_prefill", "la_prefill_varlen", "la_decode", "la_backward",
             "la_status_string", "la_read_device_status", "la_set_tuning", "la_get_tuning",
-            "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection"]
+            "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection",
+            "la_prefill_with_state", "la_prefill_varlen_with_state"]
 
 _lib = None
 
@@ -49,6 +50,9 @@ def lib():
         L.la_workspace_bytes.restype = SZ
         L.la_prefill.argtypes = [P, P, P, P, P, P, I, I, LL, I, I, I, P, SZ, P]
         L.la_prefill_varlen.argtypes = [P, I, P, P, P, P, P, P, I, LL, I, I, I, P, SZ, P]
+        L.la_prefill_with_state.argtypes = [P, P, P, P, P, P, P, I, I, LL, I, I, I, P, SZ, P]
+        L.la_prefill_varlen_with_state.argtypes = [P, I, P, P, P, P, P, P, P, I, LL, I, I, I, P,
+                                                   SZ, P]
         L.la_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
         L.la_backward.argtypes = [P, P, P, P, P, P, P, P, I, I, LL, I, I, I, P, SZ, P]
         L.la_status_string.argtypes = [I]
@@ -59,7 +63,8 @@ def lib():
         L.la_last_launch_count.argtypes = []
         L.la_prefill_noalloc.argtypes = [P, P, P, P, P, P, I, I, LL, I, I, I, P]
         L.la_set_fault_injection.argtypes = [I, I]
-        for f in ("la_prefill", "la_prefill_varlen", "la_decode", "la_backward",
+        for f in ("la_prefill", "la_prefill_varlen", "la_prefill_with_state",
+                  "la_prefill_varlen_with_state", "la_decode", "la_backward",
                   "la_read_device_status", "la_set_tuning", "la_get_tuning",
                   "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection"):
             getattr(L, f).restype = I
@@ -119,6 +124,23 @@ def la_prefill_varlen(cu_seqlens, q, k, v, slopes, o, state_out, ws, stream=None
         _ptr(state_out), H, T, d, _dt(q), _dt(o), _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def la_prefill_with_state(q, k, v, slopes, state_in, o, state_out, ws, stream=None):
+    B, H, N, d = q.shape
+    _check("la_prefill_with_state", lib().la_prefill_with_state(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(slopes), _ptr(state_in), _ptr(o), _ptr(state_out),
+        B, H, N, d, _dt(q), _dt(o), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def la_prefill_varlen_with_state(cu_seqlens, q, k, v, slopes, state_in, o, state_out, ws,
+                                 stream=None):
+    H, T, d = q.shape
+    num_seqs = cu_seqlens.numel() - 1
+    _check("la_prefill_varlen_with_state", lib().la_prefill_varlen_with_state(
+        _ptr(cu_seqlens), num_seqs, _ptr(q), _ptr(k), _ptr(v), _ptr(slopes), _ptr(state_in),
+        _ptr(o), _ptr(state_out), H, T, d, _dt(q), _dt(o), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
 def la_decode(q, k, v, slopes, state, o, stream=None):
     B, H, d = q.shape
     _check("la_decode", lib().la_decode(
@@ -172,23 +194,31 @@ def la_status_string(status) -> str:
 
 # ---------------------------------------------------------------- conveniences
 
-def prefill(q, k, v, slopes, out_dtype=None, want_state=True, stream=None):
-    """Allocate outputs and workspace, run la_prefill. Returns (O, state or None)."""
+def prefill(q, k, v, slopes, out_dtype=None, want_state=True, stream=None, state_in=None):
+    """Allocate outputs and workspace, run la_prefill (la_prefill_with_state when
+    state_in [B,H,d,d] is given). Returns (O, state or None)."""
     B, H, N, d = q.shape
     o = torch.empty_like(q, dtype=out_dtype or q.dtype)
     st = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device) if want_state else None
     ws = workspace(LA_OP_PREFILL, B, H, N, d, 0, q.dtype, q.device)
-    la_prefill(q, k, v, slopes, o, st, ws, stream)
+    if state_in is None:
+        la_prefill(q, k, v, slopes, o, st, ws, stream)
+    else:
+        la_prefill_with_state(q, k, v, slopes, state_in, o, st, ws, stream)
     return o, st
 
 
-def prefill_varlen(cu_seqlens, q, k, v, slopes, out_dtype=None, want_state=True, stream=None):
+def prefill_varlen(cu_seqlens, q, k, v, slopes, out_dtype=None, want_state=True, stream=None,
+                   state_in=None):
     H, T, d = q.shape
     S = cu_seqlens.numel() - 1
     o = torch.empty_like(q, dtype=out_dtype or q.dtype)
     st = torch.empty((S, H, d, d), dtype=torch.float32, device=q.device) if want_state else None
     ws = workspace(LA_OP_PREFILL_VARLEN, 1, H, T, d, S, q.dtype, q.device)
-    la_prefill_varlen(cu_seqlens, q, k, v, slopes, o, st, ws, stream)
+    if state_in is None:
+        la_prefill_varlen(cu_seqlens, q, k, v, slopes, o, st, ws, stream)
+    else:
+        la_prefill_varlen_with_state(cu_seqlens, q, k, v, slopes, state_in, o, st, ws, stream)
     return o, st
 
 

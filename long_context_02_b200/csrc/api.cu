@@ -89,9 +89,12 @@ LA_API size_t la_workspace_bytes(int op, int B, int H, long long N_or_total, int
     }
 }
 
-LA_API int la_prefill(const void* q, const void* k, const void* v, const float* slopes, void* o,
-                      float* state_out, int B, int H, long long N, int d, int in_t, int out_t,
-                      void* workspace, size_t ws_bytes, la_stream_t stream)
+namespace {
+
+// Dense prefill, optionally continued from per-(sequence, head) states.
+int prefill_dense(const void* q, const void* k, const void* v, const float* slopes,
+                  const float* state_in, void* o, float* state_out, int B, int H, long long N,
+                  int d, int in_t, int out_t, void* workspace, size_t ws_bytes, la_stream_t stream)
 {
     g_launches = 0;
     if (B <= 0 || H <= 0 || N < 0) return LA_ERR_INVALID_ARG;
@@ -101,7 +104,7 @@ LA_API int la_prefill(const void* q, const void* k, const void* v, const float* 
     // With N == 0 the token tensors are empty and may be NULL.
     if (!slopes || (N > 0 && (!q || !k || !v || !o))) return LA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(slopes) ||
-        (state_out && !aligned16(state_out)))
+        (state_out && !aligned16(state_out)) || !aligned16(state_in))
         return LA_ERR_INVALID_ARG;
     Problems P;
     P.H = H;
@@ -113,15 +116,16 @@ LA_API int la_prefill(const void* q, const void* k, const void* v, const float* 
     if ((st = status_of(clear_header(workspace, s))) != LA_OK) return st;
     if (use_tensor_cores(in_t, d))
         return status_of(launch_tc_forward(P, q, k, v, slopes, o, state_out, d, out_t, g_segment,
-                                           workspace, s));
+                                           workspace, s, 0, state_in));
     return status_of(launch_simt_forward(P, q, k, v, slopes, o, state_out, d, in_t, out_t,
-                                         default_block(), 0, s));
+                                         default_block(), 0, s, state_in));
 }
 
-LA_API int la_prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q, const void* k,
-                             const void* v, const float* slopes, void* o, float* state_out, int H,
-                             long long total, int d, int in_t, int out_t, void* workspace,
-                             size_t ws_bytes, la_stream_t stream)
+// Packed variable-length prefill, optionally continued from per-(sequence, head) states.
+int prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q, const void* k,
+                   const void* v, const float* slopes, const float* state_in, void* o,
+                   float* state_out, int H, long long total, int d, int in_t, int out_t,
+                   void* workspace, size_t ws_bytes, la_stream_t stream)
 {
     g_launches = 0;
     if (num_seqs < 0 || H <= 0 || total < 0) return LA_ERR_INVALID_ARG;
@@ -131,7 +135,7 @@ LA_API int la_prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q,
     if (!cu_seqlens || !slopes || (total > 0 && (!q || !k || !v || !o)))
         return LA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(slopes) ||
-        (state_out && !aligned16(state_out)) ||
+        (state_out && !aligned16(state_out)) || !aligned16(state_in) ||
         (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
         return LA_ERR_INVALID_ARG;
     Problems P;
@@ -146,9 +150,55 @@ LA_API int la_prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q,
     if (num_seqs == 0) return LA_OK;
     if (use_tensor_cores(in_t, d))
         return status_of(launch_tc_forward(P, q, k, v, slopes, o, state_out, d, out_t, g_segment,
-                                           workspace, s));
+                                           workspace, s, 0, state_in));
     return status_of(launch_simt_forward(P, q, k, v, slopes, o, state_out, d, in_t, out_t,
-                                         default_block(), 0, s));
+                                         default_block(), 0, s, state_in));
+}
+
+}  // namespace
+
+LA_API int la_prefill(const void* q, const void* k, const void* v, const float* slopes, void* o,
+                      float* state_out, int B, int H, long long N, int d, int in_t, int out_t,
+                      void* workspace, size_t ws_bytes, la_stream_t stream)
+{
+    return prefill_dense(q, k, v, slopes, nullptr, o, state_out, B, H, N, d, in_t, out_t,
+                         workspace, ws_bytes, stream);
+}
+
+LA_API int la_prefill_with_state(const void* q, const void* k, const void* v,
+                                 const float* slopes, const float* state_in, void* o,
+                                 float* state_out, int B, int H, long long N, int d, int in_t,
+                                 int out_t, void* workspace, size_t ws_bytes, la_stream_t stream)
+{
+    if (!state_in) {
+        g_launches = 0;
+        return LA_ERR_INVALID_ARG;
+    }
+    return prefill_dense(q, k, v, slopes, state_in, o, state_out, B, H, N, d, in_t, out_t,
+                         workspace, ws_bytes, stream);
+}
+
+LA_API int la_prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q, const void* k,
+                             const void* v, const float* slopes, void* o, float* state_out, int H,
+                             long long total, int d, int in_t, int out_t, void* workspace,
+                             size_t ws_bytes, la_stream_t stream)
+{
+    return prefill_varlen(cu_seqlens, num_seqs, q, k, v, slopes, nullptr, o, state_out, H, total,
+                          d, in_t, out_t, workspace, ws_bytes, stream);
+}
+
+LA_API int la_prefill_varlen_with_state(const int* cu_seqlens, int num_seqs, const void* q,
+                                        const void* k, const void* v, const float* slopes,
+                                        const float* state_in, void* o, float* state_out, int H,
+                                        long long total, int d, int in_t, int out_t,
+                                        void* workspace, size_t ws_bytes, la_stream_t stream)
+{
+    if (!state_in) {
+        g_launches = 0;
+        return LA_ERR_INVALID_ARG;
+    }
+    return prefill_varlen(cu_seqlens, num_seqs, q, k, v, slopes, state_in, o, state_out, H, total,
+                          d, in_t, out_t, workspace, ws_bytes, stream);
 }
 
 LA_API int la_decode(const void* q, const void* k, const void* v, const float* slopes,

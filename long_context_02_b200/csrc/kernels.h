@@ -21,10 +21,12 @@ struct Problems {
 // SIMT chunked forward (fp32 FFMA): the fp32 path, and the bf16 path for
 // head dims the tensor-core kernel does not take. reverse != 0 runs the
 // time-reversed operator O_i = sum_{j >= i} lam^(j-i) (q_i . k_j) v_j.
+// state_in (may be null or equal to state_out) is the state before the first
+// token of each (sequence, head).
 cudaError_t launch_simt_forward(const Problems& P, const void* q, const void* k, const void* v,
                                 const float* slopes, void* o, float* state_out, int d,
                                 int in_t, int out_t, int block, int reverse,
-                                cudaStream_t stream);
+                                cudaStream_t stream, const float* state_in = nullptr);
 
 // Fused single-token decode step.
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* slopes,

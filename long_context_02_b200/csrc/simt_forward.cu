@@ -32,6 +32,7 @@ struct SimtArgs {
     float* state_out;
     Problems P;
     int reverse;
+    const float* state_in;  // [problems][D][D] state before the first token, or null
 };
 
 template <int D, int DV, int C>
@@ -69,7 +70,11 @@ __global__ void __launch_bounds__(256) simt_forward_kernel(SimtArgs a)
     }
     const float slope = a.slopes[h];
     for (int m = threadIdx.x; m <= C; m += blockDim.x) pw[m] = expf(-slope * (float)m);
-    for (int e = threadIdx.x; e < D * DV; e += blockDim.x) Ss[e] = 0.f;
+    // The carried state starts as the caller's incoming state (or zero); this
+    // CTA reads its own column slice before it writes that slice of state_out.
+    const float* s_in = a.state_in ? a.state_in + st_idx * D * D : nullptr;
+    for (int e = threadIdx.x; e < D * DV; e += blockDim.x)
+        Ss[e] = s_in ? s_in[(e / DV) * D + c0 + e % DV] : 0.f;
 
     const Tin* q = (const Tin*)a.q + row0 * D;
     const Tin* k = (const Tin*)a.k + row0 * D;
@@ -186,9 +191,9 @@ cudaError_t launch_t(const SimtArgs& a, int d, int block, cudaStream_t stream)
 cudaError_t launch_simt_forward(const Problems& P, const void* q, const void* k, const void* v,
                                 const float* slopes, void* o, float* state_out, int d,
                                 int in_t, int out_t, int block, int reverse,
-                                cudaStream_t stream)
+                                cudaStream_t stream, const float* state_in)
 {
-    SimtArgs a{q, k, v, slopes, o, state_out, P, reverse};
+    SimtArgs a{q, k, v, slopes, o, state_out, P, reverse, reverse ? nullptr : state_in};
     if (in_t == LA_F32 && out_t == LA_F32) return launch_t<float, float>(a, d, block, stream);
     if (in_t == LA_BF16 && out_t == LA_F32)
         return launch_t<__nv_bfloat16, float>(a, d, block, stream);

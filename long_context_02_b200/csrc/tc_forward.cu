@@ -138,6 +138,7 @@ struct Params {
     const float* slopes;
     void* o;
     float* state_out;
+    const float* state_in;  // [chains][D][D] state before token 0 (null: zero), forward only
     int reverse;
     WsHeader* hdr;
     int* chain_flags;   // per (chain, half): segments published so far
@@ -1082,7 +1083,8 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
 #pragma unroll
             for (int x = 0; x < DV / 2; ++x) S[x] = 0ull;
         }
-        // Incoming state: the predecessor's inclusive prefix (zero for the first segment).
+        // Incoming state: the predecessor's inclusive prefix; for the first
+        // segment the caller's state before token 0, or zero.
         const float* src = p.incl + (((size_t)chain2 * 2 + ((it.p_ord - 1) & 1)) * D + a) * DV;
         if (it.p_ord > 0) {
             if (a == 0) {
@@ -1111,9 +1113,16 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
             const uint64_t dl2 = f2(dl, dl);
             float* dst = p.incl + (((size_t)chain2 * 2 + (it.p_ord & 1)) * D + a) * DV;
             const bool has_prev = it.p_ord > 0;
+            // The caller's state may be the state_out array itself: it is read here,
+            // before this chain's first publish, and written after the last segment.
+            const float* s_in = (has_prev || p.state_in == nullptr)
+                                    ? nullptr
+                                    : p.state_in + ((size_t)it.chain * D + a) * D + DV * it.half;
 #pragma unroll
             for (int x = 0; x < DV / 4; ++x) {
-                const float4 w = has_prev ? ld_cg_ordered(src + 4 * x) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 w = has_prev ? ld_cg_ordered(src + 4 * x)
+                                 : s_in   ? ld_cg_ordered(s_in + 4 * x)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
                 const uint64_t w0 = f2(w.x, w.y), w1 = f2(w.z, w.w);
                 if (has_succ) {
                     const uint64_t o0 = fma2(dl2, w0, S[2 * x]), o1 = fma2(dl2, w1, S[2 * x + 1]);
@@ -1228,11 +1237,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
 }
 
-// Varlen planner: segment-major list of (chain, p_ord, nseg) items; zero
-// states for empty sequences. One CTA of 1024 threads.
+// Varlen planner: segment-major list of (chain, p_ord, nseg) items; the
+// final state of an empty sequence is its incoming state (or zero). One CTA
+// of 1024 threads.
 __global__ void __launch_bounds__(1024) plan_varlen_kernel(const int* cu, int num_seqs, int H,
                                                            int seg, int4* items, int max_items,
-                                                           WsHeader* hdr, float* state_out)
+                                                           WsHeader* hdr, float* state_out,
+                                                           const float* state_in)
 {
     __shared__ int warp_tot[32];
     __shared__ int s_max;
@@ -1250,7 +1261,10 @@ __global__ void __launch_bounds__(1024) plan_varlen_kernel(const int* cu, int nu
         for (int s = 0; s < num_seqs; ++s) {
             if (cu[s + 1] - cu[s] > 0) continue;
             float4* dst = reinterpret_cast<float4*>(state_out + (size_t)s * H * D * D);
-            for (int x = tid; x < H * D * D / 4; x += blockDim.x) dst[x] = make_float4(0, 0, 0, 0);
+            const float4* src =
+                state_in ? reinterpret_cast<const float4*>(state_in + (size_t)s * H * D * D) : nullptr;
+            for (int x = tid; x < H * D * D / 4; x += blockDim.x)
+                dst[x] = src ? src[x] : make_float4(0, 0, 0, 0);
         }
     }
     __syncthreads();
@@ -1435,7 +1449,8 @@ size_t tc_workspace_bytes(const Problems& P, int d, int seg_tuning, bool varlen)
 
 cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, const void* v,
                               const float* slopes, void* o, float* state_out, int d, int out_t,
-                              int seg_tuning, void* workspace, cudaStream_t stream, int reverse)
+                              int seg_tuning, void* workspace, cudaStream_t stream, int reverse,
+                              const float* state_in)
 {
     using namespace tc;
     (void)d;
@@ -1445,8 +1460,10 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     cudaError_t err;
     if (!varlen && P.N == 0) {
-        if (state_out)
-            return cudaMemsetAsync(state_out, 0, sizeof(float) * (size_t)P.count() * D * D, stream);
+        const size_t bytes = sizeof(float) * (size_t)P.count() * D * D;
+        if (state_out && state_in && state_in != state_out)
+            return cudaMemcpyAsync(state_out, state_in, bytes, cudaMemcpyDeviceToDevice, stream);
+        if (state_out && !state_in) return cudaMemsetAsync(state_out, 0, bytes, stream);
         return cudaSuccess;
     }
     if (varlen && P.total == 0 && P.num_seqs == 0) return cudaSuccess;
@@ -1467,6 +1484,7 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     prm.slopes = slopes;
     prm.o = o;
     prm.state_out = state_out;
+    prm.state_in = reverse ? nullptr : state_in;
     prm.reverse = reverse;
     prm.hdr = reinterpret_cast<WsHeader*>(ws);
     prm.chain_flags = reinterpret_cast<int*>(ws + w.flags);
@@ -1485,7 +1503,7 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     if (varlen) {
         plan_varlen_kernel<<<1, 1024, 0, stream>>>(P.cu_seqlens, P.num_seqs, P.H, seg,
                                                     const_cast<int4*>(prm.items), (int)w.max_items,
-                                                    prm.hdr, state_out);
+                                                    prm.hdr, state_out, prm.state_in);
         count_launch();
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         if (P.total == 0) return cudaSuccess;

@@ -20,11 +20,12 @@ extern FaultInjection g_fault;
 size_t tc_workspace_bytes(const Problems& P, int d, int seg_tuning, bool varlen);
 
 // Forward prefill (dense or varlen). reverse != 0 runs the time-reversed
-// operator (used by the backward pass).
+// operator (used by the backward pass). state_in (forward only, may be null or
+// equal to state_out): per (sequence, head) state before the first token.
 cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, const void* v,
                               const float* slopes, void* o, float* state_out, int d, int out_t,
                               int seg_tuning, void* workspace, cudaStream_t stream,
-                              int reverse = 0);
+                              int reverse = 0, const float* state_in = nullptr);
 
 // Backward: dQ by the forward operator on (dO, V, K); dK and dV by the
 // time-reversed operator on (V, dO, Q) and (K, Q, dO).

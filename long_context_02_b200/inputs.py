@@ -98,6 +98,14 @@ def decode_inputs(B, H, d, dtype=torch.bfloat16, device="cpu", seed=0, state_sig
     return q, k, v, state, slopes(H, device)
 
 
+def state_inputs(B, H, d, device="cpu", seed=0, sigma=0.5):
+    """An incoming state [B,H,d,d] fp32 with entries ~ N(0, sigma^2) (the state of
+    a cached prefix; sigma 0.5 is the order of the slow heads' states under the
+    prefill workloads' inputs)."""
+    g = _gen(seed, device)
+    return torch.randn((B, H, d, d), generator=g, device=device) * sigma
+
+
 def grad_output(shape, dtype=torch.bfloat16, device="cpu", seed=1):
     """dO ~ N(0,1)."""
     g = _gen(seed, device)

@@ -105,6 +105,24 @@ def test_varlen_argument_errors(lib):
                                  None) == B.LA_ERR_INVALID_ARG
 
 
+def test_with_state_argument_errors(lib):
+    P = ctypes.c_void_p
+    x = P(16)
+    # the incoming state is required and must be 16-byte aligned
+    assert lib.la_prefill_with_state(x, x, x, x, None, x, x, 1, 2, 64, 64, 1, 1, x, 1 << 20,
+                                     None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_prefill_with_state(x, x, x, x, P(20), x, x, 1, 2, 64, 64, 1, 1, x, 1 << 20,
+                                     None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_prefill_with_state(x, x, x, x, x, x, x, 0, 2, 64, 64, 1, 1, x, 1 << 20,
+                                     None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_prefill_with_state(x, x, x, x, x, x, x, 1, 2, 64, 64, 1, 1, None, 0,
+                                     None) == B.LA_ERR_WORKSPACE
+    assert lib.la_prefill_varlen_with_state(x, 2, x, x, x, x, None, x, None, 4, 100, 128, 0, 0,
+                                            x, 1 << 30, None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_prefill_varlen_with_state(None, 2, x, x, x, x, x, x, None, 4, 100, 128, 0, 0,
+                                            x, 1 << 30, None) == B.LA_ERR_INVALID_ARG
+
+
 def test_tuning_roundtrip(lib):
     assert lib.la_set_tuning(48, 0) == B.LA_ERR_INVALID_ARG
     assert lib.la_set_tuning(0, 100) == B.LA_ERR_INVALID_ARG

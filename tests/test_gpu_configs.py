@@ -60,6 +60,24 @@ def test_minimax_prefill_32k():
         assert np.max(np.abs(got - want)) <= TOL_BF16 * rms, f"rows of head {h}"
 
 
+def test_minimax_prefill_32k_with_state():
+    """The 32K prefill continued from an incoming state, in place (the launch
+    bench.py times for the cached-prefix leg)."""
+    B, H, N, d = 1, 64, 32768, 128
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.bfloat16, DEV, seed=1002)
+    s_in = inputs.state_inputs(B, H, d, DEV, seed=1003)
+    st = s_in.clone()
+    o = torch.empty(q.shape, dtype=torch.float32, device=DEV)
+    ws = L.workspace(L.LA_OP_PREFILL, B, H, N, d)
+    L.la_prefill_with_state(q, k, v, s, st, o, st, ws)
+    assert L.la_read_device_status(ws) == L.LA_OK
+    hs = [0, 63]
+    o_ref, st_ref = oracle.recurrence(_heads(q, hs), _heads(k, hs), _heads(v, hs), lam(s)[hs],
+                                      state_in=f64(s_in)[:, hs])
+    assert_close(_heads(o, hs), o_ref, TOL_BF16, "O (heads 0, 63)")
+    assert_close(f64(st)[:, hs], st_ref, TOL_BF16, "state (heads 0, 63)")
+
+
 def test_varlen_16_sequences():
     H, d = 64, 128
     lengths = inputs.varlen_lengths(16, 1024, 65536, seed=0)
