@@ -220,11 +220,12 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     L.lib()  # fails loudly when the library is missing
     pk, pk_kind = peaks()
+    N = args.seq_len
 
-    q, k, v, s = inputs.prefill_inputs(B_, H_, N_, D_, torch.bfloat16, dev, seed=1000 + rank)
+    q, k, v, s = inputs.prefill_inputs(B_, H_, N, D_, torch.bfloat16, dev, seed=1000 + rank)
     o = torch.empty_like(q)
     st = torch.empty((B_, H_, D_, D_), dtype=torch.float32, device=dev)
-    ws = L.workspace(L.LA_OP_PREFILL, B_, H_, N_, D_, 0, torch.bfloat16, dev)
+    ws = L.workspace(L.LA_OP_PREFILL, B_, H_, N, D_, 0, torch.bfloat16, dev)
 
     def step():
         L.la_prefill(q, k, v, s, o, st, ws)
@@ -239,13 +240,13 @@ def run_ours(args):
     clocks = sampler.stop()
     assert L.la_read_device_status(ws) == L.LA_OK
 
-    F = prefill_flops(B_, H_, N_)
-    Bytes = prefill_bytes(B_, H_, N_)
+    F = prefill_flops(B_, H_, N)
+    Bytes = prefill_bytes(B_, H_, N)
     value = world * F / (ms * 1e-3) / 1e12  # ms is already the max over ranks
     achieved = Bytes / (ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4),
-                "traffic": profiled_traffic(), "peak_source": pk_kind,
+                "traffic": profiled_traffic() if N == N_ else None, "peak_source": pk_kind,
                 "kernel": "tc_forward_kernel", "algorithmic_bytes": Bytes}
 
     # End to end through the C ABI with host buffers: H2D of Q,K,V from pinned
@@ -260,7 +261,7 @@ def run_ours(args):
         hst = torch.empty(st.shape, dtype=st.dtype).pin_memory()
         groups = 8
         hg = H_ // groups
-        ws_g = L.workspace(L.LA_OP_PREFILL, B_, hg, N_, D_, 0, torch.bfloat16, dev)
+        ws_g = L.workspace(L.LA_OP_PREFILL, B_, hg, N, D_, 0, torch.bfloat16, dev)
         s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
 
         def e2e_step():
@@ -306,16 +307,17 @@ def run_ours(args):
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded: Q,K = SiLU(N(0,1))/sqrt(d), V = N(0,1))",
-        "config": {"workload": "MiniMax-shaped prefill B=1 H=64 N=32768 d=128 bf16",
-                   "B": B_, "H": H_, "N": N_, "d": D_, "global_batch": B_ * world,
-                   "seq_len": N_, "out_dtype": "bf16", "state": "fp32",
+        "config": {"workload": f"MiniMax-shaped prefill B=1 H=64 N={N} d=128 bf16",
+                   "B": B_, "H": H_, "N": N, "d": D_, "global_batch": B_ * world,
+                   "seq_len": N, "out_dtype": "bf16", "state": "fp32",
                    "parallelism": f"replicas x{world} (independent heads, no collective)",
-                   "l2": "inputs (1.5 GB per step) larger than the 126 MB L2; no flush",
+                   "l2": (f"inputs ({3 * q.numel() * 2 / 1e9:.2f} GB per step) larger than the "
+                          "126 MB L2; no flush"),
                    "flop_convention": "B*H*N*(4d^2 + 4*256*d)"},
-        "tokens_per_s": round(world * B_ * N_ / (ms * 1e-3), 1),
-        "token_heads_per_s": round(world * B_ * H_ * N_ / (ms * 1e-3), 1),
+        "tokens_per_s": round(world * B_ * N / (ms * 1e-3), 1),
+        "token_heads_per_s": round(world * B_ * H_ * N / (ms * 1e-3), 1),
         "pct_tensor_peak": round(100 * value / world / pk["bf16_tflops"], 2),
-        "tflops_executed": round(world * B_ * H_ * N_ * (4 * D_ * D_ * 1.25 + 4 * 128 * D_)
+        "tflops_executed": round(world * B_ * H_ * N * (4 * D_ * D_ * 1.25 + 4 * 128 * D_)
                                  / (ms * 1e-3) / 1e12, 3),
         "roofline": roofline,
         "cpu_baseline": cpu,
@@ -329,6 +331,42 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def bench_mixed(L, inputs, dev, world, steps):
+    """A batch of 20 cached inputs, two of 50 tokens and 18 of one token (the
+    shape of the separated prefill/decode example in section 3.3 of the
+    MiniMax-01 summary), H=64, d=128: la_mixed_step with prefill and decode on
+    two streams, on one stream, and the whole batch through the prefill kernel."""
+    lengths = [1] * 20
+    lengths[3] = lengths[11] = 50
+    H, d, S = 64, 128, len(lengths)
+    q, k, v, cu, s = inputs.varlen_inputs(lengths, H, d, torch.bfloat16, dev, seed=17)
+    T = q.shape[1]
+    st = inputs.state_inputs(S, H, d, dev, seed=18)
+    o = torch.empty_like(q)
+    ws = L.workspace(L.LA_OP_PREFILL_VARLEN, 1, H, T, d, S, torch.bfloat16, dev)
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream(device=dev)
+
+    def two():
+        side.wait_stream(main)
+        L.la_mixed_step(cu, q, k, v, s, st, o, ws, main, side)
+        main.wait_stream(side)
+
+    legs = {"two_streams": two,
+            "one_stream": lambda: L.la_mixed_step(cu, q, k, v, s, st, o, ws, main, main),
+            "prefill_kernel_only":
+                lambda: L.la_prefill_varlen_with_state(cu, q, k, v, s, st, o, st, ws)}
+    res = {"workload": "20 cached inputs (2 x 50 tokens, 18 x 1 token) H=64 d=128 bf16, "
+                       "fp32 states advanced in place"}
+    n = max(20, steps)
+    for name, fn in legs.items():
+        for _ in range(3):
+            fn()
+        res[name + "_us"] = round(1e3 * timed(fn, n, world), 2)
+    del q, k, v, st, o, ws
+    return res
 
 
 def run_secondary(args, L, inputs, dev, world, pk):
@@ -380,6 +418,7 @@ def run_secondary(args, L, inputs, dev, world, pk):
         "ms": round(ms, 4), "TFLOP/s": round(world * F / (ms * 1e-3) / 1e12, 2),
         "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
     del q, k, v, st, o, ws
+    out["mixed"] = bench_mixed(L, inputs, dev, world, steps)
     if not args.quick:
         # varlen: 16 sequences of U{1024..65536} tokens, packed
         lengths = inputs.varlen_lengths(16, 1024, 65536, seed=0)
@@ -499,6 +538,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="skip the varlen and long legs")
+    ap.add_argument("--seq-len", type=int, default=N_,
+                    help="tokens of the headline prefill (default: the MiniMax-shaped 32768)")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

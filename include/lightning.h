@@ -156,6 +156,34 @@ LA_API int la_decode(const void* q, const void* k, const void* v, const float* s
                      la_stream_t stream);
 
 /*
+ * One step over a batch of cached inputs of mixed lengths, with prefill and
+ * decoding separated ("MiniMax-01 ... | Summary", section 3.3, Separated
+ * Prefill and Decoding Execution: single-token inputs and longer inputs go to
+ * different kernels on separate CUDA streams). Sequence s of the packed batch
+ * continues from its state states[s] and covers tokens
+ * [cu_seqlens[s], cu_seqlens[s+1]):
+ *   - one-token sequences: the decode step (la_decode) on decode_stream;
+ *   - longer sequences: the prefill from their states
+ *     (la_prefill_varlen_with_state) on prefill_stream;
+ *   - empty sequences: nothing (their states stay as they are).
+ * The result is that of la_prefill_varlen_with_state over the whole batch.
+ *   cu_seqlens  in      device int32 [num_seqs + 1] (as for la_prefill_varlen)
+ *   q, k, v     in      [H][total][d], dtype in_t
+ *   states      in/out  [num_seqs][H][d][d] fp32, advanced in place
+ *   o           out     [H][total][d], dtype out_t
+ *   workspace   at least la_workspace_bytes(LA_OP_PREFILL_VARLEN, ...) bytes;
+ *               used on prefill_stream only (read its device status there)
+ * The two parts touch disjoint rows and states. The call orders neither
+ * stream after the other: the caller makes both wait for the work that
+ * produced the inputs and waits for both before reading the outputs. The
+ * streams may be the same stream (then the parts run one after the other).
+ */
+LA_API int la_mixed_step(const int* cu_seqlens, int num_seqs, const void* q, const void* k,
+                         const void* v, const float* slopes, float* states, void* o, int H,
+                         long long total, int d, int in_t, int out_t, void* workspace,
+                         size_t ws_bytes, la_stream_t prefill_stream, la_stream_t decode_stream);
+
+/*
  * Gradients of L = <dO, O> with respect to q, k and v for [B][H][N][d]
  * inputs (the pages state no backward pass; these are the derivatives of the
  * operator above):

@@ -201,6 +201,43 @@ LA_API int la_prefill_varlen_with_state(const int* cu_seqlens, int num_seqs, con
                           d, in_t, out_t, workspace, ws_bytes, stream);
 }
 
+LA_API int la_mixed_step(const int* cu_seqlens, int num_seqs, const void* q, const void* k,
+                         const void* v, const float* slopes, float* states, void* o, int H,
+                         long long total, int d, int in_t, int out_t, void* workspace,
+                         size_t ws_bytes, la_stream_t prefill_stream, la_stream_t decode_stream)
+{
+    g_launches = 0;
+    if (num_seqs < 0 || H <= 0 || total < 0) return LA_ERR_INVALID_ARG;
+    int st = check_d(d);
+    if (st != LA_OK) return st;
+    if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;
+    if (!cu_seqlens || !slopes || !states || (total > 0 && (!q || !k || !v || !o)))
+        return LA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(slopes) ||
+        !aligned16(states) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return LA_ERR_INVALID_ARG;
+    Problems P;
+    P.H = H;
+    P.num_seqs = num_seqs;
+    P.cu_seqlens = cu_seqlens;
+    P.total = total;
+    P.min_len = 2;  // one-token sequences go to the decode kernel
+    if ((st = check_workspace(workspace, ws_bytes, workspace_for(P, d, in_t, true))) != LA_OK)
+        return st;
+    cudaStream_t ps = reinterpret_cast<cudaStream_t>(prefill_stream);
+    cudaStream_t ds = reinterpret_cast<cudaStream_t>(decode_stream);
+    if ((st = status_of(clear_header(workspace, ps))) != LA_OK) return st;
+    if (num_seqs == 0) return LA_OK;
+    cudaError_t e = use_tensor_cores(in_t, d)
+                        ? launch_tc_forward(P, q, k, v, slopes, o, states, d, out_t, g_segment,
+                                            workspace, ps, 0, states)
+                        : launch_simt_forward(P, q, k, v, slopes, o, states, d, in_t, out_t,
+                                              default_block(), 0, ps, states);
+    if (e != cudaSuccess) return LA_ERR_CUDA;
+    return status_of(launch_decode_packed(cu_seqlens, num_seqs, q, k, v, slopes, states, o, H,
+                                          total, d, in_t, out_t, ds));
+}
+
 LA_API int la_decode(const void* q, const void* k, const void* v, const float* slopes,
                      float* state_inout, void* o, int B, int H, int d, int in_t, int out_t,
                      la_stream_t stream)

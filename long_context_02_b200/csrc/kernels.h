@@ -15,6 +15,8 @@ struct Problems {
     int num_seqs = 0;               // dense: B; varlen: number of sequences
     const int* cu_seqlens = nullptr;  // varlen when not null
     long long total = 0;            // varlen: packed length
+    int min_len = 1;                // varlen: sequences shorter than this (but not empty)
+                                    // are left alone (outputs and states untouched)
     long long count() const { return (long long)num_seqs * H; }
 };
 
@@ -32,5 +34,12 @@ cudaError_t launch_simt_forward(const Problems& P, const void* q, const void* k,
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* slopes,
                           float* state, void* o, int B, int H, int d, int in_t, int out_t,
                           cudaStream_t stream);
+
+// The decode step for the one-token sequences of a packed [H][total][d]
+// batch (states [num_seqs][H][d][d]); every other sequence is left alone.
+cudaError_t launch_decode_packed(const int* cu_seqlens, int num_seqs, const void* q,
+                                 const void* k, const void* v, const float* slopes,
+                                 float* states, void* o, int H, long long total, int d, int in_t,
+                                 int out_t, cudaStream_t stream);
 
 }  // namespace la

@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(256) simt_forward_kernel(SimtArgs a)
         const long long b = a.P.cu_seqlens[s], e = a.P.cu_seqlens[s + 1];
         row0 = (long long)h * a.P.total + b;
         len = e - b;
+        if (len > 0 && len < a.P.min_len) return;  // served by another kernel
         st_idx = prob;  // s * H + h
     } else {
         row0 = prob * a.P.N;

@@ -1238,19 +1238,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // Varlen planner: segment-major list of (chain, p_ord, nseg) items; the
-// final state of an empty sequence is its incoming state (or zero). One CTA
-// of 1024 threads.
+// final state of an empty sequence is its incoming state (or zero).
+// Sequences with 0 < length < min_len get no items (another kernel serves
+// them). One CTA of 1024 threads.
 __global__ void __launch_bounds__(1024) plan_varlen_kernel(const int* cu, int num_seqs, int H,
                                                            int seg, int4* items, int max_items,
                                                            WsHeader* hdr, float* state_out,
-                                                           const float* state_in)
+                                                           const float* state_in, int min_len)
 {
     __shared__ int warp_tot[32];
     __shared__ int s_max;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     auto nseg_of = [&](int s) -> int {
         const long long L = (long long)cu[s + 1] - cu[s];
-        return L > 0 ? (int)((L + seg - 1) / seg) : 0;
+        return L > 0 && L >= min_len ? (int)((L + seg - 1) / seg) : 0;
     };
     if (tid == 0) s_max = 0;
     __syncthreads();
@@ -1278,7 +1279,7 @@ __global__ void __launch_bounds__(1024) plan_varlen_kernel(const int* cu, int nu
         __syncthreads();
         for (int s = tid; s < num_seqs; s += blockDim.x) {
             const long long Ls = len_of(s);
-            if (Ls <= 0) continue;
+            if (Ls <= 0 || Ls < min_len) continue;
             atomicAdd(&s_count, 1);
             int rank = 0;
             for (int s2 = 0; s2 < num_seqs; ++s2) {
@@ -1503,7 +1504,7 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     if (varlen) {
         plan_varlen_kernel<<<1, 1024, 0, stream>>>(P.cu_seqlens, P.num_seqs, P.H, seg,
                                                     const_cast<int4*>(prm.items), (int)w.max_items,
-                                                    prm.hdr, state_out, prm.state_in);
+                                                    prm.hdr, state_out, prm.state_in, P.min_len);
         count_launch();
         if ((err = cudaGetLastError()) != cudaSuccess) return err;
         if (P.total == 0) return cudaSuccess;

@@ -123,6 +123,20 @@ def test_with_state_argument_errors(lib):
                                             x, 1 << 30, None) == B.LA_ERR_INVALID_ARG
 
 
+def test_mixed_step_argument_errors(lib):
+    P = ctypes.c_void_p
+    x = P(16)
+    # states are required; the workspace is that of the varlen prefill
+    assert lib.la_mixed_step(x, 2, x, x, x, x, None, x, 4, 100, 128, 0, 0, x, 1 << 30, None,
+                             None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_mixed_step(None, 2, x, x, x, x, x, x, 4, 100, 128, 0, 0, x, 1 << 30, None,
+                             None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_mixed_step(x, 2, x, x, x, x, x, x, 4, 100, 96, 0, 0, x, 1 << 30, None,
+                             None) == B.LA_ERR_UNSUPPORTED
+    assert lib.la_mixed_step(x, 2, x, x, x, x, x, x, 4, 100, 128, 0, 0, x, 64, None,
+                             None) == B.LA_ERR_WORKSPACE
+
+
 def test_tuning_roundtrip(lib):
     assert lib.la_set_tuning(48, 0) == B.LA_ERR_INVALID_ARG
     assert lib.la_set_tuning(0, 100) == B.LA_ERR_INVALID_ARG
