@@ -94,9 +94,10 @@ class Oracle:
         lib.oracle_recurrence.argtypes = [I, P, P, P, P, P, P, P, P, P, P, L, I]
         lib.oracle_backward.argtypes = [I, P, P, P, P, P, P, P, P, P, P, L]
         lib.oracle_decode.argtypes = [P, P, P, P, P, P, L, L]
+        lib.oracle_norm_gate.argtypes = [P, P, P, D, P, L, L, L, L]
         lib.oracle_forward_rows.argtypes = [P, P, P, P, L, P, L, D]
         for f in ("oracle_forward", "oracle_forward_from_state", "oracle_recurrence", "oracle_backward", "oracle_decode",
-                  "oracle_forward_rows"):
+                  "oracle_forward_rows", "oracle_norm_gate"):
             getattr(lib, f).restype = None
         self.lib = lib
 
@@ -179,6 +180,15 @@ class Oracle:
         self.lib.oracle_decode(_p(q), _p(k), _p(v), _p(lp), _p(st), _p(o), B * H, d)
         return o, st
 
+    def norm_gate(self, o, g, w, eps):
+        """RMS normalization over the H*d features of each token, then a sigmoid
+        gate. o [B,H,N,d] (head-major); g [B,N,H*d]; w [H*d]. Returns Y [B,N,H*d]."""
+        o, g, w = _f64(o), _f64(g), _f64(w)
+        B, H, N, d = o.shape
+        y = _out((B, N, H * d))
+        self.lib.oracle_norm_gate(_p(o), _p(g), _p(w), float(eps), _p(y), B, H, N, d)
+        return y
+
     def backward(self, dout, q, k, v, lam):
         """Quadratic-sum gradients of <dO, O>, all [B,H,N,d]. Returns (dQ, dK, dV)."""
         dout, q, k, v = _f64(dout), _f64(q), _f64(k), _f64(v)
@@ -236,6 +246,10 @@ def decode(*a, **kw):
 
 def backward(*a, **kw):
     return default().backward(*a, **kw)
+
+
+def norm_gate(*a, **kw):
+    return default().norm_gate(*a, **kw)
 
 
 def backward_recurrence(*a, **kw):

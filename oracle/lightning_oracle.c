@@ -177,6 +177,39 @@ void oracle_decode(const double* q, const double* k, const double* v, const doub
     }
 }
 
+/* Output normalization and gate after the operator ("MiniMax-01: Scaling
+ * Foundation Models with Lightning Attention | Summary", section 2.2: the
+ * linear-attention output passes through Norm, and the blocks use gating; the
+ * page gives neither form). Read as an RMS normalization over all H*d
+ * features of a token followed by a sigmoid gate:
+ *
+ *   r_{b,n}         = 1 / sqrt( (1/(H d)) sum_{h,c} O[b][h][n][c]^2 + eps )
+ *   Y[b][n][h d + c] = w[h d + c] * O[b][h][n][c] * r_{b,n} * sigmoid(G[b][n][h d + c])
+ *
+ * O is head-major [B][H][N][d]; G, w and Y are token-major [B][N][H d]. */
+void oracle_norm_gate(const double* o, const double* g, const double* w, double eps,
+                      double* y, long B, long H, long N, long d)
+{
+    #pragma omp parallel for schedule(static)
+    for (long t = 0; t < B * N; ++t) {
+        long b = t / N, n = t % N;
+        double ss = 0.0;
+        for (long h = 0; h < H; ++h)
+            for (long c = 0; c < d; ++c) {
+                double x = o[((b * H + h) * N + n) * d + c];
+                ss += x * x;
+            }
+        double r = 1.0 / sqrt(ss / (double)(H * d) + eps);
+        for (long h = 0; h < H; ++h)
+            for (long c = 0; c < d; ++c) {
+                long f = h * d + c;
+                double x = o[((b * H + h) * N + n) * d + c];
+                double gate = 1.0 / (1.0 + exp(-g[t * H * d + f]));
+                y[t * H * d + f] = w[f] * x * r * gate;
+            }
+    }
+}
+
 /* Gradients of <dO, O> for (1), each by its own quadratic sum:
  *   dQ_i = sum_{j <= i} lam^(i-j) (dO_i . v_j) k_j
  *   dK_j = sum_{i >= j} lam^(i-j) (dO_i . v_j) q_i

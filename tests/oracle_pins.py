@@ -20,6 +20,10 @@ What pins what:
   cutting a sequence and carrying the state  -> forward / recurrence with state_in
   all-ones closed form with a constant state -> forward with state_in
   varlen with states == per-sequence calls   -> forward_varlen with state_in
+  hand fixture (tests/golden/norm_gate_hand.txt) -> norm_gate (axis, layout, gate)
+  constant rows closed form                  -> norm_gate (eps)
+  unit rms after the norm                    -> norm_gate (the mean over H*d)
+  scale invariance                           -> norm_gate
 """
 from __future__ import annotations
 
@@ -346,6 +350,54 @@ def pin_state_in_varlen_is_per_sequence(orc, seed=11):
             np.testing.assert_allclose(st[s], st_s[0], rtol=1e-13, atol=1e-14)
 
 
+def pin_norm_gate_hand_fixture(orc):
+    path = os.path.join(GOLDEN, "norm_gate_hand.txt")
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *nums = line.split()
+            g3 = np.log(3.0)
+            vals[key] = np.array([g3 if x == "g3" else -g3 if x == "-g3" else float(x)
+                                  for x in nums])
+    y = orc.norm_gate(vals["O"].reshape(1, 2, 2, 2), vals["G"].reshape(1, 2, 4), vals["w"],
+                      float(vals["eps"][0]))
+    np.testing.assert_allclose(y.reshape(-1), vals["Y"], rtol=1e-14, atol=0)
+
+
+def pin_norm_gate_constant_rows(orc):
+    """O = c everywhere, G = 0, w = 1: Y = c / sqrt(c^2 + eps) / 2."""
+    B, H, N, d, c, eps = 2, 3, 5, 4, 3.0, 0.25
+    o = np.full((B, H, N, d), c)
+    y = orc.norm_gate(o, np.zeros((B, N, H * d)), np.ones(H * d), eps)
+    np.testing.assert_allclose(y, np.full((B, N, H * d), c / np.sqrt(c * c + eps) / 2),
+                               rtol=1e-14)
+
+
+def pin_norm_gate_unit_rms(orc, seed=12):
+    """eps = 0, w = 1 and a saturated gate: every token's Y has mean square 1
+    over its H*d features."""
+    rng = np.random.default_rng(seed)
+    B, H, N, d = 2, 4, 7, 8
+    o = rng.standard_normal((B, H, N, d)) * rng.uniform(0.1, 10, size=(B, H, N, 1))
+    y = orc.norm_gate(o, np.full((B, N, H * d), 50.0), np.ones(H * d), 0.0)
+    np.testing.assert_allclose(np.mean(y * y, axis=2), 1.0, rtol=1e-13)
+
+
+def pin_norm_gate_scale_invariance(orc, seed=13):
+    """Y(a O, a^2 eps) = Y(O, eps)."""
+    rng = np.random.default_rng(seed)
+    B, H, N, d = 1, 3, 6, 4
+    o = rng.standard_normal((B, H, N, d))
+    g = rng.standard_normal((B, N, H * d))
+    w = rng.standard_normal(H * d)
+    a, eps = 7.25, 0.3
+    np.testing.assert_allclose(orc.norm_gate(a * o, g, w, a * a * eps),
+                               orc.norm_gate(o, g, w, eps), rtol=1e-13, atol=1e-15)
+
+
 ALL_PINS = [
     pin_hand_fixture,
     pin_rational_brute_force,
@@ -362,4 +414,8 @@ ALL_PINS = [
     pin_state_in_split_invariance,
     pin_state_in_all_ones,
     pin_state_in_varlen_is_per_sequence,
+    pin_norm_gate_hand_fixture,
+    pin_norm_gate_constant_rows,
+    pin_norm_gate_unit_rms,
+    pin_norm_gate_scale_invariance,
 ]

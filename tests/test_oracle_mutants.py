@@ -68,6 +68,24 @@ MUTANTS = [
     ("recurrence_ignores_state_in",
      "if (state_in) memcpy(S, state_in",
      "if (0) memcpy(S, state_in"),
+    ("norm_sum_of_values_not_squares",
+     "ss += x * x;",
+     "ss += x;"),
+    ("norm_mean_over_one_head",
+     "double r = 1.0 / sqrt(ss / (double)(H * d) + eps);",
+     "double r = 1.0 / sqrt(ss / (double)d + eps);"),
+    ("norm_drops_eps",
+     "double r = 1.0 / sqrt(ss / (double)(H * d) + eps);",
+     "double r = 1.0 / sqrt(ss / (double)(H * d));"),
+    ("gate_sign_flipped",
+     "double gate = 1.0 / (1.0 + exp(-g[t * H * d + f]));",
+     "double gate = 1.0 / (1.0 + exp(g[t * H * d + f]));"),
+    ("norm_gate_output_transposed",
+     "y[t * H * d + f] = w[f] * x * r * gate;",
+     "y[t * H * d + c * H + h] = w[f] * x * r * gate;"),
+    ("norm_gate_reads_o_token_major",
+     "double x = o[((b * H + h) * N + n) * d + c];\n                double gate",
+     "double x = o[t * H * d + f];\n                double gate"),
     ("varlen_zero_length_state_not_cleared",
      "if (st) for (long a = 0; a < d * d; ++a) st[a] = 0.0;\n            continue;",
      "continue;"),
