@@ -419,6 +419,21 @@ def run_secondary(args, L, inputs, dev, world, pk):
         "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
     del q, k, v, st, o, ws
     out["mixed"] = bench_mixed(L, inputs, dev, world, steps)
+    # output normalization and gate on the prefill's output (bf16 O, gate and Y)
+    o = torch.randn((1, 64, 32768, 128), device=dev).to(torch.bfloat16)
+    g = torch.randn((1, 32768, 64 * 128), device=dev).to(torch.bfloat16)
+    w = torch.ones(64 * 128, device=dev)
+    y = torch.empty_like(g)
+    fn = lambda: L.la_output_norm_gate(o, g, w, 1e-5, y)
+    for _ in range(3):
+        fn()
+    ms = timed(fn, steps, world)
+    nbytes = 3 * o.numel() * 2
+    out["norm_gate"] = {"workload": "RMS norm over H*d + sigmoid gate, B=1 H=64 N=32768 d=128 bf16",
+                        "ms": round(ms, 4), "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                        "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                        "bytes": nbytes}
+    del o, g, w, y
     if not args.quick:
         # varlen: 16 sequences of U{1024..65536} tokens, packed
         lengths = inputs.varlen_lengths(16, 1024, 65536, seed=0)

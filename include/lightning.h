@@ -184,6 +184,25 @@ LA_API int la_mixed_step(const int* cu_seqlens, int num_seqs, const void* q, con
                          size_t ws_bytes, la_stream_t prefill_stream, la_stream_t decode_stream);
 
 /*
+ * Output normalization and gate, the step after the operator ("MiniMax-01 ...
+ * | Summary", section 2.2: the linear-attention output passes through a
+ * normalization, and the blocks gate it; the page gives neither form). This
+ * library takes an RMS normalization over all H*d features of a token and a
+ * sigmoid gate, and turns the head-major output into token-major rows:
+ *     r_{b,n}          = 1 / sqrt( mean_{h,c} O[b][h][n][c]^2 + eps )
+ *     Y[b][n][h d + c] = w[h d + c] * O[b][h][n][c] * r_{b,n} * sigmoid(G[b][n][h d + c])
+ *   o       in   [B][H][N][d], dtype o_t (the prefill's output; varlen: B = 1, N = total)
+ *   gate    in   [B][N][H*d], dtype y_t
+ *   weight  in   [H*d] fp32
+ *   eps     in   >= 0 and finite
+ *   y       out  [B][N][H*d], dtype y_t; must not overlap o or gate
+ * LA_ERR_UNSUPPORTED when H*d > 16384. No workspace; N may be 0.
+ */
+LA_API int la_output_norm_gate(const void* o, const void* gate, const float* weight, float eps,
+                               void* y, int B, int H, long long N, int d, int o_t, int y_t,
+                               la_stream_t stream);
+
+/*
  * Gradients of L = <dO, O> with respect to q, k and v for [B][H][N][d]
  * inputs (the pages state no backward pass; these are the derivatives of the
  * operator above):

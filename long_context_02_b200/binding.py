@@ -26,7 +26,8 @@ LA_OP_PREFILL, LA_OP_PREFILL_VARLEN, LA_OP_DECODE, LA_OP_BACKWARD = 0, 1, 2, 3
 EXPORTED = ["la_workspace_bytes", "la_prefill", "la_prefill_varlen", "la_decode", "la_backward",
             "la_status_string", "la_read_device_status", "la_set_tuning", "la_get_tuning",
             "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection",
-            "la_prefill_with_state", "la_prefill_varlen_with_state", "la_mixed_step"]
+            "la_prefill_with_state", "la_prefill_varlen_with_state", "la_mixed_step",
+            "la_output_norm_gate"]
 
 _lib = None
 
@@ -55,6 +56,7 @@ def lib():
                                                    SZ, P]
         L.la_mixed_step.argtypes = [P, I, P, P, P, P, P, P, I, LL, I, I, I, P, SZ, P, P]
         L.la_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+        L.la_output_norm_gate.argtypes = [P, P, P, ctypes.c_float, P, I, I, LL, I, I, I, P]
         L.la_backward.argtypes = [P, P, P, P, P, P, P, P, I, I, LL, I, I, I, P, SZ, P]
         L.la_status_string.argtypes = [I]
         L.la_status_string.restype = ctypes.c_char_p
@@ -65,7 +67,8 @@ def lib():
         L.la_prefill_noalloc.argtypes = [P, P, P, P, P, P, I, I, LL, I, I, I, P]
         L.la_set_fault_injection.argtypes = [I, I]
         for f in ("la_prefill", "la_prefill_varlen", "la_prefill_with_state",
-                  "la_prefill_varlen_with_state", "la_mixed_step", "la_decode", "la_backward",
+                  "la_prefill_varlen_with_state", "la_mixed_step", "la_output_norm_gate",
+                  "la_decode", "la_backward",
                   "la_read_device_status", "la_set_tuning", "la_get_tuning",
                   "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection"):
             getattr(L, f).restype = I
@@ -150,6 +153,13 @@ def la_mixed_step(cu_seqlens, q, k, v, slopes, states, o, ws, prefill_stream=Non
         _ptr(cu_seqlens), num_seqs, _ptr(q), _ptr(k), _ptr(v), _ptr(slopes), _ptr(states),
         _ptr(o), H, T, d, _dt(q), _dt(o), _ptr(ws), ws.numel(), _stream(prefill_stream),
         _stream(decode_stream)))
+
+
+def la_output_norm_gate(o, gate, weight, eps, y, stream=None):
+    B, H, N, d = o.shape
+    _check("la_output_norm_gate", lib().la_output_norm_gate(
+        _ptr(o), _ptr(gate), _ptr(weight), float(eps), _ptr(y), B, H, N, d, _dt(o), _dt(y),
+        _stream(stream)))
 
 
 def la_decode(q, k, v, slopes, state, o, stream=None):

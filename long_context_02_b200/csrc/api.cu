@@ -238,6 +238,25 @@ LA_API int la_mixed_step(const int* cu_seqlens, int num_seqs, const void* q, con
                                           total, d, in_t, out_t, ds));
 }
 
+LA_API int la_output_norm_gate(const void* o, const void* gate, const float* weight, float eps,
+                               void* y, int B, int H, long long N, int d, int o_t, int y_t,
+                               la_stream_t stream)
+{
+    g_launches = 0;
+    if (B <= 0 || H <= 0 || N < 0) return LA_ERR_INVALID_ARG;
+    int st = check_d(d);
+    if (st != LA_OK) return st;
+    if ((o_t != LA_BF16 && o_t != LA_F32) || (y_t != LA_BF16 && y_t != LA_F32))
+        return LA_ERR_INVALID_ARG;
+    if (!(eps >= 0.f) || eps > 3.0e38f) return LA_ERR_INVALID_ARG;  // also rejects NaN
+    if (!norm_gate_supported(H, d)) return LA_ERR_UNSUPPORTED;
+    if (N > 0 && (!o || !gate || !weight || !y)) return LA_ERR_INVALID_ARG;
+    if (!aligned16(o) || !aligned16(gate) || !aligned16(weight) || !aligned16(y))
+        return LA_ERR_INVALID_ARG;
+    return status_of(launch_norm_gate(o, gate, weight, eps, y, B, H, N, d, o_t, y_t,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 LA_API int la_decode(const void* q, const void* k, const void* v, const float* slopes,
                      float* state_inout, void* o, int B, int H, int d, int in_t, int out_t,
                      la_stream_t stream)

@@ -35,6 +35,13 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
                           float* state, void* o, int B, int H, int d, int in_t, int out_t,
                           cudaStream_t stream);
 
+// Output normalization and gate (RMS over each token's H*d features, then a
+// sigmoid gate); O head-major [B][H][N][d], G and Y token-major [B][N][H*d].
+bool norm_gate_supported(int H, int d);
+cudaError_t launch_norm_gate(const void* o, const void* g, const float* w, float eps, void* y,
+                             int B, int H, long long N, int d, int o_t, int g_t,
+                             cudaStream_t stream);
+
 // The decode step for the one-token sequences of a packed [H][total][d]
 // batch (states [num_seqs][H][d][d]); every other sequence is left alone.
 cudaError_t launch_decode_packed(const int* cu_seqlens, int num_seqs, const void* q,

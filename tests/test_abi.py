@@ -137,6 +137,26 @@ def test_mixed_step_argument_errors(lib):
                              None) == B.LA_ERR_WORKSPACE
 
 
+def test_norm_gate_argument_errors(lib):
+    P = ctypes.c_void_p
+    x = P(16)
+    f = ctypes.c_float
+    assert lib.la_output_norm_gate(x, x, x, f(1e-5), x, 1, 129, 10, 128, 0, 0,
+                                   None) == B.LA_ERR_UNSUPPORTED   # H*d > 16384
+    assert lib.la_output_norm_gate(x, x, x, f(-1.0), x, 1, 4, 10, 128, 0, 0,
+                                   None) == B.LA_ERR_INVALID_ARG   # eps < 0
+    assert lib.la_output_norm_gate(x, x, x, f(float("nan")), x, 1, 4, 10, 128, 0, 0,
+                                   None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_output_norm_gate(x, None, x, f(1e-5), x, 1, 4, 10, 128, 0, 0,
+                                   None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_output_norm_gate(x, x, P(24), f(1e-5), x, 1, 4, 10, 128, 0, 0,
+                                   None) == B.LA_ERR_INVALID_ARG   # misaligned weight
+    assert lib.la_output_norm_gate(x, x, x, f(1e-5), x, 1, 4, 10, 96, 0, 0,
+                                   None) == B.LA_ERR_UNSUPPORTED
+    assert lib.la_output_norm_gate(x, x, x, f(1e-5), x, 1, 4, 10, 128, 0, 5,
+                                   None) == B.LA_ERR_INVALID_ARG
+
+
 def test_tuning_roundtrip(lib):
     assert lib.la_set_tuning(48, 0) == B.LA_ERR_INVALID_ARG
     assert lib.la_set_tuning(0, 100) == B.LA_ERR_INVALID_ARG
