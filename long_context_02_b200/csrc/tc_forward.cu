@@ -367,16 +367,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return r;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
-
-// x0, x1 -> (hi, lo) bf16x2 words with x = hi + lo to about 2^-16 relative.
-__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo)
-{
-    hi = pack_bf16x2(x0, x1);
-    lo = pack_bf16x2(x0 - bf16_lo(hi), x1 - bf16_hi(hi));
-}
-
 // Pairs of fp32 in one 64-bit register for the packed f32x2 instructions.
 __device__ __forceinline__ uint64_t f2(float a, float b)
 {
@@ -426,27 +416,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
 {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// K-major 128 x 128 tile (two 64-column boxes): k-step ks covers K elements [16ks, 16ks+16).
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int ks)
-{
-    return sdesc(tile + (uint32_t)(ks >> 2) * BOX_BYTES + (uint32_t)(ks & 3) * 32u, 16u, 1024u);
-}
-
-// MN-major tile with rows = K dim and two 64-element boxes along MN,
-// BOX_BYTES apart (the leading byte offset): k-step ks covers rows
-// [16ks, 16ks+16).
-__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int ks)
-{
-    return sdesc(tile + (uint32_t)ks * 2048u, BOX_BYTES, 1024u);
-}
-
-// MN-major box, 64 elements wide (one swizzle atom along MN, so the leading
-// byte offset is not used; it is kept small and in bounds).
-__device__ __forceinline__ uint64_t desc_mn64(uint32_t box, int ks)
-{
-    return sdesc(box + (uint32_t)ks * 2048u, 16u, 1024u);
 }
 
 __device__ __forceinline__ int num_blocks(int len) { return (len + C - 1) / C; }
