@@ -95,9 +95,10 @@ class Oracle:
         lib.oracle_backward.argtypes = [I, P, P, P, P, P, P, P, P, P, P, L]
         lib.oracle_decode.argtypes = [P, P, P, P, P, P, L, L]
         lib.oracle_norm_gate.argtypes = [P, P, P, D, P, L, L, L, L]
+        lib.oracle_state_prefix.argtypes = [P, P, P, L, L, L, L, P]
         lib.oracle_forward_rows.argtypes = [P, P, P, P, L, P, L, D]
         for f in ("oracle_forward", "oracle_forward_from_state", "oracle_recurrence", "oracle_backward", "oracle_decode",
-                  "oracle_forward_rows", "oracle_norm_gate"):
+                  "oracle_forward_rows", "oracle_norm_gate", "oracle_state_prefix"):
             getattr(lib, f).restype = None
         self.lib = lib
 
@@ -189,6 +190,18 @@ class Oracle:
         self.lib.oracle_norm_gate(_p(o), _p(g), _p(w), float(eps), _p(y), B, H, N, d)
         return y
 
+    def state_prefix(self, states, lam, lens, r):
+        """Incoming state of chunk r from the local states of consecutive chunks.
+        states [R,B,H,d,d] (each chunk's own state); lam [H]; lens [R].
+        Returns [B,H,d,d]."""
+        states = _f64(states)
+        R, B, H, d, _ = states.shape
+        lp = _f64(np.tile(np.asarray(lam, dtype=np.float64).reshape(-1), B))
+        ln = _i64(lens)
+        out = _out((B, H, d, d))
+        self.lib.oracle_state_prefix(_p(states), _p(lp), _p(ln), R, int(r), B * H, d, _p(out))
+        return out
+
     def backward(self, dout, q, k, v, lam):
         """Quadratic-sum gradients of <dO, O>, all [B,H,N,d]. Returns (dQ, dK, dV)."""
         dout, q, k, v = _f64(dout), _f64(q), _f64(k), _f64(v)
@@ -250,6 +263,10 @@ def backward(*a, **kw):
 
 def norm_gate(*a, **kw):
     return default().norm_gate(*a, **kw)
+
+
+def state_prefix(*a, **kw):
+    return default().state_prefix(*a, **kw)
 
 
 def backward_recurrence(*a, **kw):

@@ -177,6 +177,36 @@ void oracle_decode(const double* q, const double* k, const double* v, const doub
     }
 }
 
+/* Incoming state of chunk r of a sequence cut into R consecutive chunks, from
+ * the chunks' local states ("MiniMax-01: Scaling Foundation Models with
+ * Lightning Attention | Summary", section 3.2, LASP+: every partition
+ * summarizes its keys and values locally, the summaries are gathered, and
+ * each partition builds its global prefix from them). Chunk p of length n_p
+ * has local state S_p (the state of its tokens alone) and decay alpha_p =
+ * lam^n_p over its whole length; the state after chunks 0..r-1 is
+ *
+ *   S_in(r) = sum_{p<r} ( prod_{p<q<r} alpha_q ) S_p
+ *
+ * evaluated here as that sum, with the product taken as lam raised to the
+ * total length of the chunks strictly between p and r.
+ * states: [R][nprob][d][d]; lam: [nprob]; lens: [R]; out: [nprob][d][d]. */
+void oracle_state_prefix(const double* states, const double* lam, const long* lens, long R,
+                         long r, long nprob, long d, double* out)
+{
+    for (long x = 0; x < nprob; ++x) {
+        double* o = out + x * d * d;
+        for (long e = 0; e < d * d; ++e) o[e] = 0.0;
+        for (long p = 0; p < r; ++p) {
+            long between = 0;
+            for (long q = p + 1; q < r; ++q) between += lens[q];
+            double w = pow(lam[x], (double)between);
+            const double* S = states + (p * nprob + x) * d * d;
+            for (long e = 0; e < d * d; ++e) o[e] += w * S[e];
+        }
+    }
+    (void)R;
+}
+
 /* Output normalization and gate after the operator ("MiniMax-01: Scaling
  * Foundation Models with Lightning Attention | Summary", section 2.2: the
  * linear-attention output passes through Norm, and the blocks use gating; the

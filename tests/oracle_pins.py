@@ -24,6 +24,8 @@ What pins what:
   constant rows closed form                  -> norm_gate (eps)
   unit rms after the norm                    -> norm_gate (the mean over H*d)
   scale invariance                           -> norm_gate
+  chunk states combine to the prefix's state -> state_prefix
+  exact rational chunks                      -> state_prefix
 """
 from __future__ import annotations
 
@@ -398,6 +400,36 @@ def pin_norm_gate_scale_invariance(orc, seed=13):
                                orc.norm_gate(o, g, w, eps), rtol=1e-13, atol=1e-15)
 
 
+def pin_state_prefix_split(orc, seed=14):
+    """Cut a sequence into chunks of unequal length: combining the chunks'
+    local states gives, for every r, the state of chunks 0..r-1 taken as one
+    sequence (the quadratic form over the concatenation)."""
+    rng = np.random.default_rng(seed)
+    B, H, d = 1, 3, 5
+    lens = [7, 1, 0, 12, 4]
+    N = sum(lens)
+    q, k, v = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    lam = np.array([0.5, 0.9, 0.999])
+    cuts = np.concatenate([[0], np.cumsum(lens)])
+    states = np.stack([orc.forward(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], lam)[1]
+                       for a, b in zip(cuts[:-1], cuts[1:])])
+    for r in range(len(lens) + 1):
+        got = orc.state_prefix(states, lam, lens, r)
+        _, want = orc.forward(q[:, :, :cuts[r]], k[:, :, :cuts[r]], v[:, :, :cuts[r]], lam)
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-13)
+
+
+def pin_state_prefix_exact(orc):
+    """lam = 1/2 and small integer chunk states: S_in(3) = lam^(n1+n2) S0 +
+    lam^n2 S1 + S2 exactly, written out for three chunks."""
+    S = np.arange(3 * 4, dtype=np.float64).reshape(3, 1, 1, 2, 2) - 5
+    lens = [3, 2, 1]
+    got = orc.state_prefix(S, np.array([0.5]), lens, 3)[0, 0]
+    want = 0.5 ** 3 * S[0, 0, 0] + 0.5 ** 1 * S[1, 0, 0] + S[2, 0, 0]
+    assert np.array_equal(got, want), (got, want)
+    assert np.array_equal(orc.state_prefix(S, np.array([0.5]), lens, 0)[0, 0], np.zeros((2, 2)))
+
+
 ALL_PINS = [
     pin_hand_fixture,
     pin_rational_brute_force,
@@ -418,4 +450,6 @@ ALL_PINS = [
     pin_norm_gate_constant_rows,
     pin_norm_gate_unit_rms,
     pin_norm_gate_scale_invariance,
+    pin_state_prefix_split,
+    pin_state_prefix_exact,
 ]

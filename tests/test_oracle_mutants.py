@@ -86,6 +86,15 @@ MUTANTS = [
     ("norm_gate_reads_o_token_major",
      "double x = o[((b * H + h) * N + n) * d + c];\n                double gate",
      "double x = o[t * H * d + f];\n                double gate"),
+    ("state_prefix_includes_own_chunk_decay",
+     "for (long q = p + 1; q < r; ++q) between += lens[q];",
+     "for (long q = p; q < r; ++q) between += lens[q];"),
+    ("state_prefix_includes_chunk_r",
+     "for (long p = 0; p < r; ++p) {\n            long between",
+     "for (long p = 0; p <= r && p < R; ++p) {\n            long between"),
+    ("state_prefix_decay_from_the_front",
+     "for (long q = p + 1; q < r; ++q) between += lens[q];",
+     "for (long q = 0; q < p; ++q) between += lens[q];"),
     ("varlen_zero_length_state_not_cleared",
      "if (st) for (long a = 0; a < d * d; ++a) st[a] = 0.0;\n            continue;",
      "continue;"),
