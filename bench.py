@@ -419,6 +419,26 @@ def run_secondary(args, L, inputs, dev, world, pk):
         "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
     del q, k, v, st, o, ws
     out["mixed"] = bench_mixed(L, inputs, dev, world, steps)
+    # one rank's step of a sequence-parallel prefill: the 32K x 64 workload cut into
+    # 8 chunks of 4096 tokens, the last rank's chunk; the gather returns the
+    # already-gathered states (the NCCL all-gather of 8 x 4 MiB is not timed here)
+    from long_context_02_b200 import sp
+    R, n = 8, 32768 // 8
+    q, k, v, s = inputs.prefill_inputs(1, 64, n, 128, torch.bfloat16, dev, seed=19)
+    o = torch.empty_like(q)
+    st = torch.empty((1, 64, 128, 128), dtype=torch.float32, device=dev)
+    states = inputs.state_inputs(R, 64, 128, dev, seed=20).reshape(R, 1, 64, 128, 128)
+    ws = L.workspace(L.LA_OP_PREFILL, 1, 64, n, 128, 0, torch.bfloat16, dev)
+    fn = lambda: sp.sp_prefill(q, k, v, s, [n] * R, R - 1, o, st, lambda _: states, ws)
+    for _ in range(3):
+        fn()
+    ms = timed(fn, steps, world)
+    out["sp_rank_step"] = {
+        "workload": "sequence-parallel prefill, one rank of 8: 4096-token chunk of the "
+                    "H=64 d=128 bf16 32K workload (local prefill, prefix of 8 states, "
+                    "prefill from that state; all-gather not included)",
+        "ms": round(ms, 4)}
+    del q, k, v, o, st, states, ws
     # output normalization and gate on the prefill's output (bf16 O, gate and Y)
     o = torch.randn((1, 64, 32768, 128), device=dev).to(torch.bfloat16)
     g = torch.randn((1, 32768, 64 * 128), device=dev).to(torch.bfloat16)

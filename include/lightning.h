@@ -183,6 +183,29 @@ LA_API int la_mixed_step(const int* cu_seqlens, int num_seqs, const void* q, con
                          long long total, int d, int in_t, int out_t, void* workspace,
                          size_t ws_bytes, la_stream_t prefill_stream, la_stream_t decode_stream);
 
+/* Most chunks (ranks) la_state_prefix takes. */
+#define LA_MAX_CHUNKS 64
+
+/*
+ * Global prefix of a sequence-parallel prefill ("MiniMax-01 ... | Summary",
+ * section 3.2, LASP+: the sequence is cut into R consecutive chunks, one per
+ * rank; each rank summarizes its chunk locally, the summaries are gathered
+ * (one all-gather), and each rank builds the state before its chunk). With
+ * S_p the state of chunk p alone (la_prefill's state_out on that chunk) and
+ * n_p its length:
+ *     out = S_in(r) = sum_{p<r} lam^(n_{p+1} + ... + n_{r-1}) S_p
+ * the state after chunks 0..r-1, which la_prefill_with_state then continues
+ * from for chunk r (r = 0 gives zeros; r = R gives the whole sequence's state).
+ *   states  in   [R][B][H][d][d] fp32 device, the gathered local states
+ *   slopes  in   [H] fp32 device
+ *   lens    in   HOST int64 [R], chunk lengths (>= 0)
+ *   R, r    1 <= R <= LA_MAX_CHUNKS, 0 <= r <= R
+ *   out     out  [B][H][d][d] fp32 device, must not overlap states
+ * No workspace.
+ */
+LA_API int la_state_prefix(const float* states, const float* slopes, const long long* lens, int R,
+                           int r, int B, int H, int d, float* out, la_stream_t stream);
+
 /*
  * Output normalization and gate, the step after the operator ("MiniMax-01 ...
  * | Summary", section 2.2: the linear-attention output passes through a

@@ -13,7 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liblightning.so")
 SOURCES = ["api.cu", "simt_forward.cu", "decode.cu", "tc_forward.cu", "noalloc.cu",
-           "norm_gate.cu"]
+           "norm_gate.cu", "lasp.cu"]
 HEADERS = ["common.cuh", "kernels.h", "tc_forward.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

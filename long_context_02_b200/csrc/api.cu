@@ -257,6 +257,21 @@ LA_API int la_output_norm_gate(const void* o, const void* gate, const float* wei
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+LA_API int la_state_prefix(const float* states, const float* slopes, const long long* lens, int R,
+                           int r, int B, int H, int d, float* out, la_stream_t stream)
+{
+    g_launches = 0;
+    if (B <= 0 || H <= 0 || R < 1 || R > LA_MAX_CHUNKS || r < 0 || r > R) return LA_ERR_INVALID_ARG;
+    int st = check_d(d);
+    if (st != LA_OK) return st;
+    if (!states || !slopes || !lens || !out) return LA_ERR_INVALID_ARG;
+    if (!aligned16(states) || !aligned16(slopes) || !aligned16(out)) return LA_ERR_INVALID_ARG;
+    for (int p = 0; p < R; ++p)
+        if (lens[p] < 0) return LA_ERR_INVALID_ARG;
+    return status_of(launch_state_prefix(states, slopes, lens, R, r, B, H, d, out,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 LA_API int la_decode(const void* q, const void* k, const void* v, const float* slopes,
                      float* state_inout, void* o, int B, int H, int d, int in_t, int out_t,
                      la_stream_t stream)

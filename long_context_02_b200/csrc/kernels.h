@@ -35,6 +35,12 @@ cudaError_t launch_decode(const void* q, const void* k, const void* v, const flo
                           float* state, void* o, int B, int H, int d, int in_t, int out_t,
                           cudaStream_t stream);
 
+// Incoming state of chunk r of a sequence-parallel prefill from the chunks'
+// gathered local states [R][B][H][d][d] (R <= LA_MAX_CHUNKS).
+cudaError_t launch_state_prefix(const float* states, const float* slopes, const long long* lens,
+                                int R, int r, int B, int H, int d, float* out,
+                                cudaStream_t stream);
+
 // Output normalization and gate (RMS over each token's H*d features, then a
 // sigmoid gate); O head-major [B][H][N][d], G and Y token-major [B][N][H*d].
 bool norm_gate_supported(int H, int d);

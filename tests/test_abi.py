@@ -157,6 +157,27 @@ def test_norm_gate_argument_errors(lib):
                                    None) == B.LA_ERR_INVALID_ARG
 
 
+def test_state_prefix_argument_errors(lib):
+    P = ctypes.c_void_p
+    x = P(16)
+    lens = (ctypes.c_longlong * 3)(4, 5, 6)
+    bad = (ctypes.c_longlong * 3)(4, -1, 6)
+    assert lib.la_state_prefix(x, x, lens, 3, 4, 1, 2, 128, x, None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_state_prefix(x, x, lens, 0, 0, 1, 2, 128, x, None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_state_prefix(x, x, lens, 65, 1, 1, 2, 128, x, None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_state_prefix(x, x, bad, 3, 1, 1, 2, 128, x, None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_state_prefix(x, x, None, 3, 1, 1, 2, 128, x, None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_state_prefix(x, x, lens, 3, 1, 1, 2, 96, x, None) == B.LA_ERR_UNSUPPORTED
+
+
+def test_sp_prefill_checks_chunk_lengths():
+    from long_context_02_b200 import sp
+    import torch
+    q = torch.zeros((1, 2, 5, 64))
+    with pytest.raises(ValueError):
+        sp.sp_prefill(q, q, q, None, [4, 5], 0, q, None, gather=lambda s: s)
+
+
 def test_tuning_roundtrip(lib):
     assert lib.la_set_tuning(48, 0) == B.LA_ERR_INVALID_ARG
     assert lib.la_set_tuning(0, 100) == B.LA_ERR_INVALID_ARG

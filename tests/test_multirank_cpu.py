@@ -1,10 +1,13 @@
-"""The multi-GPU bench path on CPU: two gloo ranks (127.0.0.1).
+"""The multi-rank paths on CPU: two gloo ranks (127.0.0.1).
 
 bench.py runs one replica of the workload per rank (the work shards by
 independent heads and sequences, no collective on the data path) and reports
 the whole-job rate as all ranks' units over the slowest rank's time. These
 tests run that aggregation, and the reference arm's rank rule (rank 0 alone
-prints), with world size 2 on the gloo backend.
+prints), with world size 2 on the gloo backend. They also run the one
+exchange of the sequence-parallel prefill (sp.nccl_gather, the all-gather of
+the chunks' local states) and check each rank's incoming state built from
+the gathered states against the prefix it stands for.
 """
 import json
 import os
@@ -75,3 +78,47 @@ def test_reference_arm_line(tmp_path):
     assert line["impl"] == "reference" and line["unit"] == "TFLOP/s"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _sp_rank_main(rank, world, port, out):
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from long_context_02_b200 import sp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    rng = np.random.default_rng(0)                 # same sequence on every rank
+    B, H, d, lens = 1, 2, 4, [5, 9]
+    N = sum(lens)
+    q, k, v = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    lam = np.array([0.6, 0.95])
+    a = sum(lens[:rank])
+    b = a + lens[rank]
+    _, s_loc = oracle.forward(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], lam)
+    states = sp.nccl_gather()(torch.from_numpy(s_loc))   # the exchange under test
+    s_in = oracle.state_prefix(states.numpy(), lam, lens, rank)
+    _, want = oracle.forward(q[:, :, :a], k[:, :, :a], v[:, :, :a], lam)
+    ok = tuple(states.shape) == (world, B, H, d, d) and np.allclose(s_in, want, rtol=1e-12,
+                                                                    atol=1e-12)
+    out.put((rank, bool(ok)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_sequence_parallel_exchange_two_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sp_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res == [(0, True), (1, True)]
