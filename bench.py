@@ -418,6 +418,21 @@ def run_secondary(args, L, inputs, dev, world, pk):
         "ms": round(ms, 4), "TFLOP/s": round(world * F / (ms * 1e-3) / 1e12, 2),
         "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
     del q, k, v, st, o, ws
+    # final state alone (a prefix to cache, or a chunk's local state): K, V in, state out
+    q, k, v, s = inputs.prefill_inputs(1, 64, 32768, 128, torch.bfloat16, dev, seed=21)
+    del q
+    st = torch.empty((1, 64, 128, 128), dtype=torch.float32, device=dev)
+    ws = L.workspace(L.LA_OP_PREFILL, 1, 64, 32768, 128, 0, torch.bfloat16, dev)
+    fn = lambda: L.la_prefill_state(k, v, s, None, st, ws)
+    for _ in range(3):
+        fn()
+    ms = timed(fn, steps, world)
+    nbytes = 2 * k.numel() * 2 + st.numel() * 4
+    out["prefill_state_only"] = {
+        "workload": "final state only, B=1 H=64 N=32768 d=128 bf16 (K, V in; state out)",
+        "ms": round(ms, 4), "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+        "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)}
+    del k, v, st, ws
     out["mixed"] = bench_mixed(L, inputs, dev, world, steps)
     # one rank's step of a sequence-parallel prefill: the 32K x 64 workload cut into
     # 8 chunks of 4096 tokens, the last rank's chunk; the gather returns the

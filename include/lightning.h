@@ -91,6 +91,24 @@ LA_API int la_prefill(const void* q, const void* k, const void* v, const float* 
                       void* workspace, size_t ws_bytes, la_stream_t stream);
 
 /*
+ * The final state alone, without outputs: the state of a prefix to cache
+ * ("MiniMax-01 ... | Summary", section 3: cached prefixes that later inputs
+ * continue from), or a chunk's local state in a sequence-parallel prefill
+ * (section 3.2, LASP+). For every (sequence, head):
+ *     state = lam^N S_in + sum_j lam^(N-1-j) k_j^T v_j
+ *   k, v       in   [B][H][N][d], dtype in_t (no queries are needed)
+ *   state_in   in   [B][H][d][d] fp32, or NULL for a zero state; may be the
+ *                   same array as state_out
+ *   state_out  out  [B][H][d][d] fp32, not NULL
+ *   workspace  at least la_workspace_bytes(LA_OP_PREFILL, ...) bytes
+ * Errors as for la_prefill. On the bf16 path it costs the state-update part
+ * of a prefill: K and V are read once, no scores are formed.
+ */
+LA_API int la_prefill_state(const void* k, const void* v, const float* slopes,
+                            const float* state_in, float* state_out, int B, int H, long long N,
+                            int d, int in_t, void* workspace, size_t ws_bytes, la_stream_t stream);
+
+/*
  * Prefill over packed variable-length sequences ("MiniMax-01 ... | Summary",
  * section 3.2: data packing concatenates samples; the state restarts at every
  * sample boundary). Sequence s covers tokens [cu_seqlens[s], cu_seqlens[s+1])

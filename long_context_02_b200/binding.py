@@ -27,7 +27,7 @@ EXPORTED = ["la_workspace_bytes", "la_prefill", "la_prefill_varlen", "la_decode"
             "la_status_string", "la_read_device_status", "la_set_tuning", "la_get_tuning",
             "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection",
             "la_prefill_with_state", "la_prefill_varlen_with_state", "la_mixed_step",
-            "la_output_norm_gate", "la_state_prefix"]
+            "la_output_norm_gate", "la_state_prefix", "la_prefill_state"]
 
 _lib = None
 
@@ -56,6 +56,7 @@ def lib():
                                                    SZ, P]
         L.la_mixed_step.argtypes = [P, I, P, P, P, P, P, P, I, LL, I, I, I, P, SZ, P, P]
         L.la_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+        L.la_prefill_state.argtypes = [P, P, P, P, P, I, I, LL, I, I, P, SZ, P]
         L.la_state_prefix.argtypes = [P, P, ctypes.POINTER(LL), I, I, I, I, I, P, P]
         L.la_output_norm_gate.argtypes = [P, P, P, ctypes.c_float, P, I, I, LL, I, I, I, P]
         L.la_backward.argtypes = [P, P, P, P, P, P, P, P, I, I, LL, I, I, I, P, SZ, P]
@@ -69,7 +70,7 @@ def lib():
         L.la_set_fault_injection.argtypes = [I, I]
         for f in ("la_prefill", "la_prefill_varlen", "la_prefill_with_state",
                   "la_prefill_varlen_with_state", "la_mixed_step", "la_output_norm_gate",
-                  "la_state_prefix",
+                  "la_state_prefix", "la_prefill_state",
                   "la_decode", "la_backward",
                   "la_read_device_status", "la_set_tuning", "la_get_tuning",
                   "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection"):
@@ -169,6 +170,13 @@ def la_state_prefix(states, slopes, lens, r, out, stream=None):
     arr = (ctypes.c_longlong * R)(*[int(x) for x in lens])
     _check("la_state_prefix", lib().la_state_prefix(
         _ptr(states), _ptr(slopes), arr, R, int(r), B, H, d, _ptr(out), _stream(stream)))
+
+
+def la_prefill_state(k, v, slopes, state_in, state_out, ws, stream=None):
+    B, H, N, d = k.shape
+    _check("la_prefill_state", lib().la_prefill_state(
+        _ptr(k), _ptr(v), _ptr(slopes), _ptr(state_in), _ptr(state_out), B, H, N, d, _dt(k),
+        _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def la_decode(q, k, v, slopes, state, o, stream=None):

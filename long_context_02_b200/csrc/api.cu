@@ -178,6 +178,35 @@ LA_API int la_prefill_with_state(const void* q, const void* k, const void* v,
                          workspace, ws_bytes, stream);
 }
 
+LA_API int la_prefill_state(const void* k, const void* v, const float* slopes,
+                            const float* state_in, float* state_out, int B, int H, long long N,
+                            int d, int in_t, void* workspace, size_t ws_bytes, la_stream_t stream)
+{
+    g_launches = 0;
+    if (B <= 0 || H <= 0 || N < 0) return LA_ERR_INVALID_ARG;
+    int st = check_d(d);
+    if (st != LA_OK) return st;
+    if (in_t != LA_BF16 && in_t != LA_F32) return LA_ERR_INVALID_ARG;
+    if (!slopes || !state_out || (N > 0 && (!k || !v))) return LA_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(slopes) || !aligned16(state_out) ||
+        !aligned16(state_in))
+        return LA_ERR_INVALID_ARG;
+    Problems P;
+    P.H = H;
+    P.num_seqs = B;
+    P.N = N;
+    if ((st = check_workspace(workspace, ws_bytes, workspace_for(P, d, in_t, false))) != LA_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = status_of(clear_header(workspace, s))) != LA_OK) return st;
+    // No query is read and no output written: k stands in for q.
+    if (use_tensor_cores(in_t, d))
+        return status_of(launch_tc_forward(P, k, k, v, slopes, nullptr, state_out, d, LA_F32,
+                                           g_segment, workspace, s, 0, state_in, 1));
+    return status_of(launch_simt_forward(P, k, k, v, slopes, nullptr, state_out, d, in_t, LA_F32,
+                                         default_block(), 0, s, state_in, 1));
+}
+
 LA_API int la_prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q, const void* k,
                              const void* v, const float* slopes, void* o, float* state_out, int H,
                              long long total, int d, int in_t, int out_t, void* workspace,

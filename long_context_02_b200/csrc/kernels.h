@@ -28,7 +28,8 @@ struct Problems {
 cudaError_t launch_simt_forward(const Problems& P, const void* q, const void* k, const void* v,
                                 const float* slopes, void* o, float* state_out, int d,
                                 int in_t, int out_t, int block, int reverse,
-                                cudaStream_t stream, const float* state_in = nullptr);
+                                cudaStream_t stream, const float* state_in = nullptr,
+                                int state_only = 0);
 
 // Fused single-token decode step.
 cudaError_t launch_decode(const void* q, const void* k, const void* v, const float* slopes,

@@ -33,6 +33,7 @@ struct SimtArgs {
     Problems P;
     int reverse;
     const float* state_in;  // [problems][D][D] state before the first token, or null
+    int state_only;         // final states only (o is not written)
 };
 
 template <int D, int DV, int C>
@@ -103,33 +104,35 @@ __global__ void __launch_bounds__(256) simt_forward_kernel(SimtArgs a)
             Vs[e] = (r < L) ? to_f32(v[(t0 + r) * D + c0 + c]) : 0.f;
         }
         __syncthreads();
-        // Intra-tile scores: As[r][c] = lam^|r-c| (q_r . k_c) on the causal side.
-        for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
-            const int r = e / C, c = e % C;
-            float w = 0.f;
-            const bool keep = r < L && c < L && (rev ? (c >= r) : (c <= r));
-            if (keep) {
-                float s = 0.f;
+        if (!a.state_only) {  // the outputs of this tile
+            // Intra-tile scores: As[r][c] = lam^|r-c| (q_r . k_c) on the causal side.
+            for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
+                const int r = e / C, c = e % C;
+                float w = 0.f;
+                const bool keep = r < L && c < L && (rev ? (c >= r) : (c <= r));
+                if (keep) {
+                    float s = 0.f;
 #pragma unroll 8
-                for (int x = 0; x < D; ++x) s = fmaf(Qs[r * (D + 1) + x], Ks[c * (D + 1) + x], s);
-                w = s * pw[rev ? (c - r) : (r - c)];
+                    for (int x = 0; x < D; ++x) s = fmaf(Qs[r * (D + 1) + x], Ks[c * (D + 1) + x], s);
+                    w = s * pw[rev ? (c - r) : (r - c)];
+                }
+                As[r * (C + 1) + c] = w;
             }
-            As[r * (C + 1) + c] = w;
-        }
-        __syncthreads();
-        // Outputs: intra product plus the decayed carried-state product.
-        for (int e = threadIdx.x; e < C * DV; e += blockDim.x) {
-            const int r = e / DV, b = e % DV;
-            if (r >= L) continue;
-            float intra = 0.f;
-            for (int c = 0; c < L; ++c) intra = fmaf(As[r * (C + 1) + c], Vs[c * DV + b], intra);
-            float inter = 0.f;
+            __syncthreads();
+            // Outputs: intra product plus the decayed carried-state product.
+            for (int e = threadIdx.x; e < C * DV; e += blockDim.x) {
+                const int r = e / DV, b = e % DV;
+                if (r >= L) continue;
+                float intra = 0.f;
+                for (int c = 0; c < L; ++c) intra = fmaf(As[r * (C + 1) + c], Vs[c * DV + b], intra);
+                float inter = 0.f;
 #pragma unroll 8
-            for (int x = 0; x < D; ++x) inter = fmaf(Qs[r * (D + 1) + x], Ss[x * DV + b], inter);
-            const float sc = pw[rev ? (L - r) : (r + 1)];
-            o[(t0 + r) * D + c0 + b] = from_f32<Tout>(fmaf(sc, inter, intra));
+                for (int x = 0; x < D; ++x) inter = fmaf(Qs[r * (D + 1) + x], Ss[x * DV + b], inter);
+                const float sc = pw[rev ? (L - r) : (r + 1)];
+                o[(t0 + r) * D + c0 + b] = from_f32<Tout>(fmaf(sc, inter, intra));
+            }
+            __syncthreads();
         }
-        __syncthreads();
         // State update: S <- lam^L S + sum_c lam^(L-1-c) k_c^T v_c (reverse: lam^c).
         for (int e = threadIdx.x; e < D * DV; e += blockDim.x) {
             const int x = e / DV, b = e % DV;
@@ -192,9 +195,10 @@ cudaError_t launch_t(const SimtArgs& a, int d, int block, cudaStream_t stream)
 cudaError_t launch_simt_forward(const Problems& P, const void* q, const void* k, const void* v,
                                 const float* slopes, void* o, float* state_out, int d,
                                 int in_t, int out_t, int block, int reverse,
-                                cudaStream_t stream, const float* state_in)
+                                cudaStream_t stream, const float* state_in, int state_only)
 {
-    SimtArgs a{q, k, v, slopes, o, state_out, P, reverse, reverse ? nullptr : state_in};
+    SimtArgs a{q, k, v, slopes, o, state_out, P, reverse, reverse ? nullptr : state_in,
+               state_only};
     if (in_t == LA_F32 && out_t == LA_F32) return launch_t<float, float>(a, d, block, stream);
     if (in_t == LA_BF16 && out_t == LA_F32)
         return launch_t<__nv_bfloat16, float>(a, d, block, stream);

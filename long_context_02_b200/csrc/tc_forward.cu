@@ -139,6 +139,8 @@ struct Params {
     void* o;
     float* state_out;
     const float* state_in;  // [chains][D][D] state before token 0 (null: zero), forward only
+    int state_only;         // final states only: every item runs phase A alone (one
+                            // segment per chain), no outputs
     int reverse;
     WsHeader* hdr;
     int* chain_flags;   // per (chain, half): segments published so far
@@ -556,8 +558,12 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
         if (!it.valid) break;
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
-        for (int pass = has_succ ? 0 : 1; pass < 2 && ok; ++pass) {
-            const uint64_t kpol = pass ? normal : keep, vpol = pass ? drop : keep;
+        // Phase A (pass 0) loads K and V; phase C (pass 1) loads Q, K and V.
+        const int last_pass = p.state_only ? 1 : 2;
+        for (int pass = (has_succ || p.state_only) ? 0 : 1; pass < last_pass && ok; ++pass) {
+            // (a state-only pass reads K and V once)
+            const bool again = pass == 0 && !p.state_only;
+            const uint64_t kpol = again ? keep : normal, vpol = again ? keep : drop;
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int y = it.y0 + block_t0(it.len, kb, p.reverse);
                 const int s = nk & 1;
@@ -675,7 +681,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
-        if (has_succ) {
+        if (has_succ || p.state_only) {
             // Phase A: DS accumulates the segment's local state over its blocks.
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int sk = nkv & 1;
@@ -698,6 +704,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             commit(B_DS_FULL);
             ++n_ds;
         }
+        if (p.state_only) continue;
         // Phase C.
         const uint32_t q0 = nq, kv0 = nkv, g0 = g;
         if (!mma1(g0, q0, kv0)) break;
@@ -797,6 +804,7 @@ __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
     Item it;
     for (uint32_t k = 0;; ++k) {
         if (!next_item(p, sm, k, it, true, lane)) break;
+        if (p.state_only) continue;  // no phase C
         const float slope = p.slopes[it.head];
         if (!group_sync(&bars[B_P_SYNC], n_sync, sm.abort, p.hdr)) break;
         pw[row] = expf(-slope * (float)row);
@@ -927,7 +935,7 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
-        if (has_succ) {
+        if (has_succ || p.state_only) {
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int t0 = block_t0(it.len, kb, REV);
                 const int L = min(C, it.len - t0);
@@ -935,6 +943,7 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
             }
             if (!ok) break;
         }
+        if (p.state_only) continue;
         auto e_v_c = [&](int kb) -> bool {
             const int L = min(C, it.len - block_t0(it.len, kb, REV));
             return e_v(slope, L, REV ? row : L - 1 - row);
@@ -1021,6 +1030,15 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         ++n_ds;
         return true;
     };
+    // Row a of this half's 64 columns of the final state.
+    auto write_state = [&](const Item& itm) {
+        if (!p.state_out) return;
+        float4* dst = reinterpret_cast<float4*>(p.state_out + ((size_t)itm.chain * D + a) * D +
+                                                DV * itm.half);
+#pragma unroll
+        for (int x = 0; x < DV / 4; ++x)
+            dst[x] = make_float4(f2x(S[2 * x]), f2y(S[2 * x]), f2x(S[2 * x + 1]), f2y(S[2 * x + 1]));
+    };
     // Hi/lo copies of the state (row a of two swizzled 128 x 64 boxes) for the next MMA3.
     auto publish_copy = [&]() -> bool {
         if (!wait_warp(&bars[B_S_FREE], (n_s & 1) ^ 1, sm.abort, p.hdr)) return false;
@@ -1046,6 +1064,23 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         const bool has_succ = it.p_ord < it.nseg - 1;
         const int chain2 = 2 * it.chain + it.half;
         bool ok = true;
+        if (p.state_only) {
+            // The chain's whole local state, plus lam^len times the incoming state.
+            if (!read_ds(0.f, false)) break;
+            if (p.state_in) {
+                const float dl = expf(-slope * (float)it.len);
+                const uint64_t dl2 = f2(dl, dl);
+                const float* s_in = p.state_in + ((size_t)it.chain * D + a) * D + DV * it.half;
+#pragma unroll
+                for (int x = 0; x < DV / 4; ++x) {
+                    const float4 w = ld_cg_ordered(s_in + 4 * x);
+                    S[2 * x] = fma2(dl2, f2(w.x, w.y), S[2 * x]);
+                    S[2 * x + 1] = fma2(dl2, f2(w.z, w.w), S[2 * x + 1]);
+                }
+            }
+            write_state(it);
+            continue;
+        }
         if (has_succ) {
             if (!read_ds(0.f, false)) break;  // S = S_loc
         } else {
@@ -1116,13 +1151,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
             if (kb + 1 < nb && !(ok = publish_copy())) break;
         }
         if (!ok) break;
-        if (it.p_ord == it.nseg - 1 && p.state_out) {
-            float4* dst = reinterpret_cast<float4*>(p.state_out + ((size_t)it.chain * D + a) * D +
-                                                    DV * it.half);
-#pragma unroll
-            for (int x = 0; x < DV / 4; ++x)
-                dst[x] = make_float4(f2x(S[2 * x]), f2y(S[2 * x]), f2x(S[2 * x + 1]), f2y(S[2 * x + 1]));
-        }
+        if (it.p_ord == it.nseg - 1) write_state(it);
     }
 }
 
@@ -1420,12 +1449,13 @@ size_t tc_workspace_bytes(const Problems& P, int d, int seg_tuning, bool varlen)
 cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, const void* v,
                               const float* slopes, void* o, float* state_out, int d, int out_t,
                               int seg_tuning, void* workspace, cudaStream_t stream, int reverse,
-                              const float* state_in)
+                              const float* state_in, int state_only)
 {
     using namespace tc;
     (void)d;
     const bool varlen = P.cu_seqlens != nullptr;
-    const int seg = choose_seg(P, seg_tuning, varlen);
+    // State only: one segment per chain (phase A needs no scan).
+    const int seg = state_only ? (1 << 30) : choose_seg(P, seg_tuning, varlen);
     const WsLayout w = layout(P, seg, varlen);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     cudaError_t err;
@@ -1455,6 +1485,7 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     prm.o = o;
     prm.state_out = state_out;
     prm.state_in = reverse ? nullptr : state_in;
+    prm.state_only = state_only;
     prm.reverse = reverse;
     prm.hdr = reinterpret_cast<WsHeader*>(ws);
     prm.chain_flags = reinterpret_cast<int*>(ws + w.flags);

@@ -5,15 +5,15 @@ section 3.2: the sequence is cut into consecutive chunks, one per rank. Each
 rank summarizes its chunk locally, the summaries are gathered in one
 all-gather, and each rank builds its global prefix from them. Here, per rank:
 
-  1. la_prefill on the rank's chunk alone gives the chunk's local state S_r;
+  1. la_prefill_state on the rank's chunk alone gives the chunk's local state
+     S_r (keys and values only, no outputs);
   2. one all-gather of the local states (4 MiB per rank at 64 heads, d = 128);
   3. la_state_prefix forms the state before the chunk from the gathered states;
   4. la_prefill_with_state computes the chunk's outputs (and, on the last rank,
      the whole sequence's final state) from that state.
 
 Every arithmetic step runs in the library's kernels; this module only orders
-the calls and moves the states between ranks. Step 1 also computes outputs
-that step 4 overwrites: a pass that forms the state alone would halve its cost.
+the calls and moves the states between ranks.
 """
 from __future__ import annotations
 
@@ -39,12 +39,11 @@ def nccl_gather(group=None) -> Callable[[torch.Tensor], torch.Tensor]:
     return gather
 
 
-def local_state(q, k, v, slopes, o_scratch, ws, stream=None) -> torch.Tensor:
-    """Step 1: the state of this rank's chunk alone, [B,H,d,d] fp32. o_scratch
-    receives outputs from a zero state (overwritten later by step 4)."""
-    B, H, _, d = q.shape
-    st = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
-    L.la_prefill(q, k, v, slopes, o_scratch, st, ws, stream)
+def local_state(k, v, slopes, ws, stream=None) -> torch.Tensor:
+    """Step 1: the state of this rank's chunk alone, [B,H,d,d] fp32."""
+    B, H, _, d = k.shape
+    st = torch.empty((B, H, d, d), dtype=torch.float32, device=k.device)
+    L.la_prefill_state(k, v, slopes, None, st, ws, stream)
     return st
 
 
@@ -75,7 +74,7 @@ def sp_prefill(q, k, v, slopes, chunk_lens: Sequence[int], rank: int, o, state_o
         raise ValueError("chunk_lens[rank] must equal this rank's chunk length")
     if ws is None:
         ws = L.workspace(L.LA_OP_PREFILL, B, H, n, d, 0, q.dtype, q.device)
-    s_loc = local_state(q, k, v, slopes, o, ws, stream)
+    s_loc = local_state(k, v, slopes, ws, stream)
     states = gather(s_loc)
     s_in = incoming_state(states, slopes, chunk_lens, rank, stream)
     L.la_prefill_with_state(q, k, v, slopes, s_in, o, state_out, ws, stream)

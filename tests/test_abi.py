@@ -178,6 +178,19 @@ def test_sp_prefill_checks_chunk_lengths():
         sp.sp_prefill(q, q, q, None, [4, 5], 0, q, None, gather=lambda s: s)
 
 
+def test_prefill_state_argument_errors(lib):
+    P = ctypes.c_void_p
+    x = P(16)
+    assert lib.la_prefill_state(x, x, x, None, None, 1, 2, 64, 128, 0, x, 1 << 30,
+                                None) == B.LA_ERR_INVALID_ARG   # no state_out
+    assert lib.la_prefill_state(x, x, x, P(20), x, 1, 2, 64, 128, 0, x, 1 << 30,
+                                None) == B.LA_ERR_INVALID_ARG   # misaligned state_in
+    assert lib.la_prefill_state(x, x, x, None, x, 1, 2, 64, 128, 0, None, 0,
+                                None) == B.LA_ERR_WORKSPACE
+    assert lib.la_prefill_state(x, x, x, None, x, 1, 2, 64, 96, 0, x, 1 << 30,
+                                None) == B.LA_ERR_UNSUPPORTED
+
+
 def test_tuning_roundtrip(lib):
     assert lib.la_set_tuning(48, 0) == B.LA_ERR_INVALID_ARG
     assert lib.la_set_tuning(0, 100) == B.LA_ERR_INVALID_ARG

@@ -49,10 +49,8 @@ def test_sp_prefill_emulated_ranks(dtype, d, tol):
     chunk = lambda x, r: x[:, :, cuts[r]:cuts[r + 1]].contiguous()
     R = len(lens)
     # what the all-gather would return: every rank's local state
-    scratch = [torch.empty((B, H, n, d), dtype=torch.float32, device=DEV) for n in lens]
     ws = [L.workspace(L.LA_OP_PREFILL, B, H, n, d, 0, dtype) for n in lens]
-    states = torch.stack([sp.local_state(chunk(q, r), chunk(k, r), chunk(v, r), s, scratch[r],
-                                         ws[r]) for r in range(R)])
+    states = torch.stack([sp.local_state(chunk(k, r), chunk(v, r), s, ws[r]) for r in range(R)])
     outs, st = [], None
     for r in range(R):
         o = torch.full((B, H, lens[r], d), float("nan"), dtype=torch.float32, device=DEV)
@@ -68,3 +66,56 @@ def test_sp_prefill_emulated_ranks(dtype, d, tol):
     o_ref, st_ref = oracle.forward(f64(q), f64(k), f64(v), lam(s))
     assert_close(np.concatenate([f64(o) for o in outs], axis=2), o_ref, tol, "O of all chunks")
     assert_close(f64(st), st_ref, tol, "final state (last rank)")
+
+
+@pytest.mark.parametrize("seg", [0, 256])
+@pytest.mark.parametrize("N", [0, 1, 129, 700, 1500])
+def test_prefill_state_only_bf16(N, seg):
+    """la_prefill_state: the final state alone, from zero and from an incoming state."""
+    B, H, d = 2, 3, 128
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.bfloat16, DEV, seed=60 + N)
+    s_in = inputs.state_inputs(B, H, d, DEV, seed=61)
+    L.la_set_tuning(0, seg)
+    try:
+        ws = L.workspace(L.LA_OP_PREFILL, B, H, N, d)
+        st0 = torch.full((B, H, d, d), float("nan"), device=DEV)
+        L.la_prefill_state(k, v, s, None, st0, ws)
+        st1 = s_in.clone()
+        L.la_prefill_state(k, v, s, st1, st1, ws)        # advanced in place
+        assert L.la_read_device_status(ws) == L.LA_OK
+    finally:
+        L.la_set_tuning(0, 0)
+    _, want0 = oracle.forward(f64(q), f64(k), f64(v), lam(s))
+    _, want1 = oracle.forward(f64(q), f64(k), f64(v), lam(s), state_in=f64(s_in))
+    if N == 0:
+        assert torch.count_nonzero(st0) == 0 and torch.equal(st1, s_in)
+        return
+    assert_close(f64(st0), want0, TOL_BF16, "state from zero")
+    assert_close(f64(st1), want1, TOL_BF16, "state from S_in")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_prefill_state_only_fp32(d):
+    B, H, N = 1, 3, 301
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.float32, DEV, seed=62)
+    s_in = inputs.state_inputs(B, H, d, DEV, seed=63)
+    ws = L.workspace(L.LA_OP_PREFILL, B, H, N, d, 0, torch.float32)
+    st = torch.full((B, H, d, d), float("nan"), device=DEV)
+    L.la_prefill_state(k, v, s, s_in, st, ws)
+    torch.cuda.synchronize()
+    _, want = oracle.forward(f64(q), f64(k), f64(v), lam(s), state_in=f64(s_in))
+    assert_close(f64(st), want, TOL_F32, "state")
+
+
+def test_prefill_state_only_minimax_size():
+    """The 32K x 64 shape, heads 0 and 63 against the oracle's recurrence."""
+    B, H, N, d = 1, 64, 32768, 128
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.bfloat16, DEV, seed=64)
+    ws = L.workspace(L.LA_OP_PREFILL, B, H, N, d)
+    st = torch.empty((B, H, d, d), device=DEV)
+    L.la_prefill_state(k, v, s, None, st, ws)
+    assert L.la_read_device_status(ws) == L.LA_OK
+    hs = [0, 63]
+    sub = lambda t: np.stack([f64(t[0, h]) for h in hs])[None]
+    _, want = oracle.recurrence(sub(q), sub(k), sub(v), lam(s)[hs], want_o=False)
+    assert_close(f64(st)[:, hs], want, TOL_BF16, "state (heads 0, 63)")
