@@ -46,6 +46,24 @@ def test_norm_gate(H, d, o_dtype, y_dtype):
     _check(y, ref, y_dtype, f"Y H={H} d={d}")
 
 
+def test_norm_gate_extreme_gates():
+    """Saturated and infinite gate inputs give gates of (about) 0 and 1; a NaN
+    gate input gives NaN in its own element and leaves the others alone."""
+    B, H, N, d = 1, 2, 3, 64
+    o, gate, w = _operands(B, H, N, d, torch.float32, torch.float32, seed=7)
+    gate[0, 0, :8] = torch.tensor([-1e4, 1e4, float("-inf"), float("inf"), -100.0, 100.0, 0.0,
+                                   float("nan")], device=DEV)
+    y = torch.empty((B, N, H * d), device=DEV)
+    L.la_output_norm_gate(o, gate, w, EPS, y)
+    torch.cuda.synchronize()
+    ref = oracle.norm_gate(f64(o), f64(gate), f64(w), EPS)
+    got = f64(y)
+    assert np.isnan(got[0, 0, 7]) and not np.isnan(got[0, 0, :7]).any()
+    assert abs(got[0, 0, 0]) < 1e-15 and abs(got[0, 0, 2]) < 1e-15
+    np.testing.assert_allclose(got[0, 0, :7], ref[0, 0, :7], rtol=1e-5, atol=1e-15)
+    assert_close(got[:, 1:], ref[:, 1:], TOL_F32, "Y (other tokens)")
+
+
 def test_norm_gate_zero_tokens():
     o = torch.empty((1, 4, 0, 128), dtype=torch.bfloat16, device=DEV)
     g = torch.empty((1, 0, 512), dtype=torch.bfloat16, device=DEV)
