@@ -119,3 +119,28 @@ def test_prefill_state_only_minimax_size():
     sub = lambda t: np.stack([f64(t[0, h]) for h in hs])[None]
     _, want = oracle.recurrence(sub(q), sub(k), sub(v), lam(s)[hs], want_o=False)
     assert_close(f64(st)[:, hs], want, TOL_BF16, "state (heads 0, 63)")
+
+
+def test_sp_prefill_minimax_size_eight_ranks():
+    """The 32K x 64 workload cut into 8 chunks of 4096 tokens (the configuration
+    bench.py times for one rank), all ranks emulated; heads 0 and 63 against the
+    oracle's recurrence over the whole sequence."""
+    B, H, N, d, R = 1, 64, 32768, 128, 8
+    n = N // R
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.bfloat16, DEV, seed=70)
+    chunk = lambda x, r: x[:, :, r * n:(r + 1) * n].contiguous()
+    ws = L.workspace(L.LA_OP_PREFILL, B, H, n, d)
+    states = torch.stack([sp.local_state(chunk(k, r), chunk(v, r), s, ws) for r in range(R)])
+    o = torch.empty((B, H, N, d), dtype=torch.float32, device=DEV)
+    st = torch.empty((B, H, d, d), dtype=torch.float32, device=DEV)
+    for r in range(R):
+        o_r = torch.empty((B, H, n, d), dtype=torch.float32, device=DEV)
+        sp.sp_prefill(chunk(q, r), chunk(k, r), chunk(v, r), s, [n] * R, r, o_r, st,
+                      lambda _: states, ws)
+        o[:, :, r * n:(r + 1) * n] = o_r
+    assert L.la_read_device_status(ws) == L.LA_OK
+    hs = [0, 63]
+    sub = lambda t: np.stack([f64(t[0, h]) for h in hs])[None]
+    o_ref, st_ref = oracle.recurrence(sub(q), sub(k), sub(v), lam(s)[hs])
+    assert_close(sub(o), o_ref, TOL_BF16, "O (heads 0, 63)")
+    assert_close(f64(st)[:, hs], st_ref, TOL_BF16, "final state (heads 0, 63)")
