@@ -691,11 +691,15 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
                 if (!ok) break;
                 ++n_vh;
                 tc_fence_after();
+                // In phase A, E_V (done: VH_READY) is the V slot's only reader; MMA4
+                // reads K and the decayed copy. Release the slot now, so that the
+                // next V load overlaps this MMA4.
+                if (elect_one()) mbar_arrive(&bars[B_VE0 + sk]);
+                __syncwarp();
                 mma4(sk, kb > 0);
                 if (elect_one()) {
                     mma_commit(&bars[B_VH_FREE]);
                     mma_commit(&bars[B_KE0 + sk]);
-                    mma_commit(&bars[B_VE0 + sk]);
                 }
                 __syncwarp();
                 ++nkv;
