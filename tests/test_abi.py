@@ -191,6 +191,40 @@ def test_prefill_state_argument_errors(lib):
                                 None) == B.LA_ERR_UNSUPPORTED
 
 
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "lightning.h"
+int main(void) {
+    size_t ws = la_workspace_bytes(LA_OP_PREFILL, 1, 64, 32768, 128, 0, LA_BF16);
+    int bad = la_prefill(0, 0, 0, 0, 0, 0, 0, 64, 32768, 128, LA_BF16, LA_BF16, 0, 0, 0);
+    printf("%zu %d\n", ws, bad);
+    return (ws > 0 && bad == LA_ERR_INVALID_ARG &&
+            strncmp(la_status_string(bad), "LA_", 3) == 0) ? 0 : 1;
+}
+"""
+
+
+def test_plain_c_program_uses_the_library(lib, tmp_path):
+    """include/lightning.h is valid C99 (no C++ needed) and a C program links
+    against liblightning.so and calls it (argument checks only: no GPU)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not found")
+    src = tmp_path / "prog.c"
+    src.write_text(C_PROGRAM)
+    libdir = os.path.dirname(B.LIB_PATH)
+    exe = tmp_path / "prog"
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                         "-I", os.path.join(ROOT, "include"), str(src), "-L", libdir,
+                         "-llightning", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stdout + run.stderr
+
+
 def test_tuning_roundtrip(lib):
     assert lib.la_set_tuning(48, 0) == B.LA_ERR_INVALID_ARG
     assert lib.la_set_tuning(0, 100) == B.LA_ERR_INVALID_ARG
