@@ -57,6 +57,15 @@ typedef enum {
 
 typedef enum { LA_BF16 = 0, LA_F32 = 1 } la_dtype;
 
+/*
+ * Size limits of every prefill, backward and mixed-step call (larger requests
+ * return LA_ERR_UNSUPPORTED before anything is launched): N, or the packed
+ * total, at most LA_MAX_TOKENS tokens (token coordinates are 32-bit in the
+ * tensor-memory copies); B*H, or num_seqs*H, at most LA_MAX_PROBLEMS.
+ */
+#define LA_MAX_TOKENS ((long long)2147483647 - 256)
+#define LA_MAX_PROBLEMS ((long long)1 << 28)
+
 typedef enum {
     LA_OP_PREFILL = 0,
     LA_OP_PREFILL_VARLEN = 1,
@@ -237,7 +246,8 @@ LA_API int la_state_prefix(const float* states, const float* slopes, const long 
  *   weight  in   [H*d] fp32
  *   eps     in   >= 0 and finite
  *   y       out  [B][N][H*d], dtype y_t; must not overlap o or gate
- * LA_ERR_UNSUPPORTED when H*d > 16384. No workspace; N may be 0.
+ * LA_ERR_UNSUPPORTED when H*d > 16384 or B*N > LA_MAX_TOKENS. No workspace;
+ * N may be 0.
  */
 LA_API int la_output_norm_gate(const void* o, const void* gate, const float* weight, float eps,
                                void* y, int B, int H, long long N, int d, int o_t, int y_t,

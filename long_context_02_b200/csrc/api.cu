@@ -35,6 +35,14 @@ static int check_d(int d)
 
 static int status_of(cudaError_t e) { return e == cudaSuccess ? LA_OK : LA_ERR_CUDA; }
 
+// Size limits: token coordinates reach the TMA engine as 32-bit integers and
+// (sequence, head) problems are counted in 32-bit work items.
+static int check_sizes(long long B_or_seqs, int H, long long tokens)
+{
+    if (tokens > LA_MAX_TOKENS || B_or_seqs * (long long)H > LA_MAX_PROBLEMS) return LA_ERR_UNSUPPORTED;
+    return LA_OK;
+}
+
 // Whether the tcgen05 tensor-core kernel takes this request.
 static bool use_tensor_cores(int in_t, int d) { return in_t == LA_BF16 && d == 128; }
 
@@ -98,6 +106,7 @@ int prefill_dense(const void* q, const void* k, const void* v, const float* slop
 {
     g_launches = 0;
     if (B <= 0 || H <= 0 || N < 0) return LA_ERR_INVALID_ARG;
+    if (check_sizes(B, H, N) != LA_OK) return LA_ERR_UNSUPPORTED;
     int st = check_d(d);
     if (st != LA_OK) return st;
     if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;
@@ -129,6 +138,7 @@ int prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q, const voi
 {
     g_launches = 0;
     if (num_seqs < 0 || H <= 0 || total < 0) return LA_ERR_INVALID_ARG;
+    if (check_sizes(num_seqs, H, total) != LA_OK) return LA_ERR_UNSUPPORTED;
     int st = check_d(d);
     if (st != LA_OK) return st;
     if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;
@@ -184,6 +194,7 @@ LA_API int la_prefill_state(const void* k, const void* v, const float* slopes,
 {
     g_launches = 0;
     if (B <= 0 || H <= 0 || N < 0) return LA_ERR_INVALID_ARG;
+    if (check_sizes(B, H, N) != LA_OK) return LA_ERR_UNSUPPORTED;
     int st = check_d(d);
     if (st != LA_OK) return st;
     if (in_t != LA_BF16 && in_t != LA_F32) return LA_ERR_INVALID_ARG;
@@ -237,6 +248,7 @@ LA_API int la_mixed_step(const int* cu_seqlens, int num_seqs, const void* q, con
 {
     g_launches = 0;
     if (num_seqs < 0 || H <= 0 || total < 0) return LA_ERR_INVALID_ARG;
+    if (check_sizes(num_seqs, H, total) != LA_OK) return LA_ERR_UNSUPPORTED;
     int st = check_d(d);
     if (st != LA_OK) return st;
     if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;
@@ -273,12 +285,14 @@ LA_API int la_output_norm_gate(const void* o, const void* gate, const float* wei
 {
     g_launches = 0;
     if (B <= 0 || H <= 0 || N < 0) return LA_ERR_INVALID_ARG;
+    if (check_sizes(B, H, N) != LA_OK) return LA_ERR_UNSUPPORTED;
     int st = check_d(d);
     if (st != LA_OK) return st;
     if ((o_t != LA_BF16 && o_t != LA_F32) || (y_t != LA_BF16 && y_t != LA_F32))
         return LA_ERR_INVALID_ARG;
     if (!(eps >= 0.f) || eps > 3.0e38f) return LA_ERR_INVALID_ARG;  // also rejects NaN
     if (!norm_gate_supported(H, d)) return LA_ERR_UNSUPPORTED;
+    if ((long long)B * N > LA_MAX_TOKENS) return LA_ERR_UNSUPPORTED;  // one CTA per token
     if (N > 0 && (!o || !gate || !weight || !y)) return LA_ERR_INVALID_ARG;
     if (!aligned16(o) || !aligned16(gate) || !aligned16(weight) || !aligned16(y))
         return LA_ERR_INVALID_ARG;
@@ -325,6 +339,7 @@ LA_API int la_backward(const void* dO, const void* q, const void* k, const void*
 {
     g_launches = 0;
     if (B <= 0 || H <= 0 || N < 0) return LA_ERR_INVALID_ARG;
+    if (check_sizes(B, H, N) != LA_OK) return LA_ERR_UNSUPPORTED;
     int st = check_d(d);
     if (st != LA_OK) return st;
     if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;

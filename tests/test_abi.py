@@ -225,6 +225,20 @@ def test_plain_c_program_uses_the_library(lib, tmp_path):
     assert run.returncode == 0, run.stdout + run.stderr
 
 
+def test_size_limits(lib):
+    P = ctypes.c_void_p
+    x = P(16)
+    too_long = (1 << 31) - 1
+    assert _prefill(lib, N=too_long) == B.LA_ERR_UNSUPPORTED
+    assert _prefill(lib, B=1 << 20, H=1 << 9) == B.LA_ERR_UNSUPPORTED   # 2^29 problems
+    assert lib.la_prefill_varlen(x, 2, x, x, x, x, x, None, 4, too_long, 128, 0, 0, x, 1 << 30,
+                                 None) == B.LA_ERR_UNSUPPORTED
+    assert lib.la_backward(x, x, x, x, x, x, x, x, 1, 2, too_long, 64, 0, 0, x, 1 << 20,
+                           None) == B.LA_ERR_UNSUPPORTED
+    assert lib.la_mixed_step(x, 2, x, x, x, x, x, x, 4, too_long, 128, 0, 0, x, 1 << 30, None,
+                             None) == B.LA_ERR_UNSUPPORTED
+
+
 def test_tuning_roundtrip(lib):
     assert lib.la_set_tuning(48, 0) == B.LA_ERR_INVALID_ARG
     assert lib.la_set_tuning(0, 100) == B.LA_ERR_INVALID_ARG
