@@ -196,7 +196,8 @@ LA_API int la_decode(const void* q, const void* k, const void* v, const float* s
  * The result is that of la_prefill_varlen_with_state over the whole batch.
  *   cu_seqlens  in      device int32 [num_seqs + 1] (as for la_prefill_varlen)
  *   q, k, v     in      [H][total][d], dtype in_t
- *   states      in/out  [num_seqs][H][d][d] fp32, advanced in place
+ *   states      in/out  [num_seqs][H][d][d] fp32, advanced in place (NULL only when
+ *                       num_seqs == 0)
  *   o           out     [H][total][d], dtype out_t
  *   workspace   at least la_workspace_bytes(LA_OP_PREFILL_VARLEN, ...) bytes;
  *               used on prefill_stream only (read its device status there)

@@ -252,7 +252,9 @@ LA_API int la_mixed_step(const int* cu_seqlens, int num_seqs, const void* q, con
     int st = check_d(d);
     if (st != LA_OK) return st;
     if ((st = check_dtypes(in_t, out_t)) != LA_OK) return st;
-    if (!cu_seqlens || !slopes || !states || (total > 0 && (!q || !k || !v || !o)))
+    // An empty batch (num_seqs == 0) has no states and may pass NULL.
+    if (!cu_seqlens || !slopes || (num_seqs > 0 && !states) ||
+        (total > 0 && (!q || !k || !v || !o)))
         return LA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(slopes) ||
         !aligned16(states) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))

@@ -135,6 +135,9 @@ def test_mixed_step_argument_errors(lib):
                              None) == B.LA_ERR_UNSUPPORTED
     assert lib.la_mixed_step(x, 2, x, x, x, x, x, x, 4, 100, 128, 0, 0, x, 64, None,
                              None) == B.LA_ERR_WORKSPACE
+    # an empty batch may pass no states (the workspace check comes next)
+    assert lib.la_mixed_step(x, 0, None, None, None, x, None, None, 4, 0, 128, 0, 0, None, 0,
+                             None, None) == B.LA_ERR_WORKSPACE
 
 
 def test_norm_gate_argument_errors(lib):

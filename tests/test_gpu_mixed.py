@@ -77,3 +77,29 @@ def test_mixed_step_bf16_output_many_heads():
                                           state_in=f64(s_in)[:, hs])
     assert_close_bf16_out(sub(o), o_ref, TOL_BF16, "bf16 O (heads 0, 31, 63)")
     assert_close(f64(st)[:, hs], st_ref, TOL_BF16, "states (heads 0, 31, 63)")
+
+
+@pytest.mark.parametrize("lengths", [[1] * 9, [0, 1, 1, 0], [2, 130, 7, 0], [300]],
+                         ids=["all_one_token", "one_token_and_empty", "no_one_token",
+                              "single_long"])
+def test_mixed_step_edge_batches(lengths):
+    """A batch where one of the two parts has nothing to do (or both)."""
+    H, d = 4, 128
+    q, k, v, cu, s = inputs.varlen_inputs(lengths, H, d, torch.bfloat16, DEV, seed=34)
+    s_in = inputs.state_inputs(len(lengths), H, d, DEV, seed=35)
+    o, st = _mixed(q, k, v, cu, s, s_in, torch.float32, True)
+    o_ref, st_ref = oracle.forward_varlen(cu.cpu().numpy(), f64(q), f64(k), f64(v), lam(s),
+                                          state_in=f64(s_in))
+    if q.shape[1] > 0:
+        assert_close(f64(o), o_ref, TOL_BF16, "O")
+    assert_close(f64(st), st_ref, TOL_BF16, "states")
+
+
+def test_mixed_step_empty_batch():
+    H, d = 4, 128
+    cu = torch.zeros(1, dtype=torch.int32, device=DEV)
+    e = torch.empty((H, 0, d), dtype=torch.bfloat16, device=DEV)
+    st = torch.empty((0, H, d, d), device=DEV)
+    ws = L.workspace(L.LA_OP_PREFILL_VARLEN, 1, H, 0, d, 0)
+    L.la_mixed_step(cu, e, e, e, inputs.slopes(H, DEV), st, e, ws)
+    torch.cuda.synchronize()
