@@ -156,8 +156,8 @@ LA_API int la_prefill_with_state(const void* q, const void* k, const void* v,
 
 /*
  * la_prefill_varlen continued from one incoming state per (sequence, head):
- *   state_in   in   [num_seqs][H][d][d] fp32, not NULL; may be the same array
- *                   as state_out
+ *   state_in   in   [num_seqs][H][d][d] fp32, not NULL unless num_seqs == 0;
+ *                   may be the same array as state_out
  * The operator per sequence is that of la_prefill_with_state; a zero-length
  * sequence's final state is its incoming state. Every other argument, result
  * and error is as for la_prefill_varlen; the workspace size is that of

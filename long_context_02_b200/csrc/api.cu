@@ -233,7 +233,7 @@ LA_API int la_prefill_varlen_with_state(const int* cu_seqlens, int num_seqs, con
                                         long long total, int d, int in_t, int out_t,
                                         void* workspace, size_t ws_bytes, la_stream_t stream)
 {
-    if (!state_in) {
+    if (!state_in && num_seqs > 0) {  // an empty batch has no states
         g_launches = 0;
         return LA_ERR_INVALID_ARG;
     }

@@ -121,6 +121,9 @@ def test_with_state_argument_errors(lib):
                                             x, 1 << 30, None) == B.LA_ERR_INVALID_ARG
     assert lib.la_prefill_varlen_with_state(None, 2, x, x, x, x, x, x, None, 4, 100, 128, 0, 0,
                                             x, 1 << 30, None) == B.LA_ERR_INVALID_ARG
+    # an empty batch may pass no states (the workspace check comes next)
+    assert lib.la_prefill_varlen_with_state(x, 0, None, None, None, x, None, None, None, 4, 0,
+                                            128, 0, 0, None, 0, None) == B.LA_ERR_WORKSPACE
 
 
 def test_mixed_step_argument_errors(lib):
