@@ -125,7 +125,8 @@ LA_API int la_prefill_state(const void* k, const void* v, const float* slopes,
  *   cu_seqlens in   device int32 [num_seqs + 1], cu_seqlens[0] = 0, non-decreasing,
  *                   cu_seqlens[num_seqs] = total (not checked: needs a device read)
  *   state_out  out  [num_seqs][H][d][d] fp32, may be NULL
- * A zero-length sequence produces no rows and a zero state.
+ * A zero-length sequence produces no rows and a zero state. num_seqs == 0 with
+ * total > 0 is LA_ERR_INVALID_ARG (tokens that belong to no sequence).
  */
 LA_API int la_prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q, const void* k,
                              const void* v, const float* slopes, void* o, float* state_out, int H,
@@ -318,8 +319,10 @@ LA_API int la_set_fault_injection(int skip_publish, int wait_limit_us);
  * plugin whose host application forbids allocations after start-up, a
  * latency-critical loop that must not call cudaMalloc).
  *
- * Same arguments, results and errors as la_prefill, minus the workspace. The
- * scratch is a fixed array of LA_NOALLOC_SCRATCH_BYTES in device memory that
+ * Same arguments, results and errors as la_prefill, minus the workspace.
+ * A device-side error of the call (a bounded wait of the state scan that gave
+ * up) is written into the built-in scratch, not into a caller's workspace:
+ * read it with la_noalloc_device_status. The scratch is a fixed array of LA_NOALLOC_SCRATCH_BYTES in device memory that
  * every GPU which loads the library holds until the process exits. Requests
  * whose la_workspace_bytes(LA_OP_PREFILL, ...) exceeds that size are refused
  * with LA_ERR_WORKSPACE before any GPU work (for bf16 inputs with d = 128 the
@@ -337,6 +340,18 @@ LA_API int la_set_fault_injection(int skip_publish, int wait_limit_us);
 LA_API int la_prefill_noalloc(const void* q, const void* k, const void* v, const float* slopes,
                               void* o, float* state_out, int B, int H, long long N, int d,
                               int in_t, int out_t, la_stream_t stream);
+
+/*
+ * Device-side status of the last la_prefill_noalloc on the current device.
+ * This is la_read_device_status for the built-in scratch, and has no
+ * counterpart on the pages either. It synchronizes `stream` (the stream the
+ * call ran on), then copies the status word out of the scratch into host
+ * memory: LA_OK, or LA_ERR_TIMEOUT when a bounded wait of the state scan gave
+ * up (that call's outputs are then invalid; the context stays usable).
+ * Returns LA_ERR_CUDA if the synchronization or the copy fails. Allocates
+ * nothing. A later la_prefill_noalloc on the device overwrites the word.
+ */
+LA_API int la_noalloc_device_status(la_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -27,7 +27,7 @@ EXPORTED = ["la_workspace_bytes", "la_prefill", "la_prefill_varlen", "la_decode"
             "la_status_string", "la_read_device_status", "la_set_tuning", "la_get_tuning",
             "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection",
             "la_prefill_with_state", "la_prefill_varlen_with_state", "la_mixed_step",
-            "la_output_norm_gate", "la_state_prefix", "la_prefill_state"]
+            "la_output_norm_gate", "la_state_prefix", "la_prefill_state", "la_noalloc_device_status"]
 
 _lib = None
 
@@ -68,12 +68,14 @@ def lib():
         L.la_last_launch_count.argtypes = []
         L.la_prefill_noalloc.argtypes = [P, P, P, P, P, P, I, I, LL, I, I, I, P]
         L.la_set_fault_injection.argtypes = [I, I]
+        L.la_noalloc_device_status.argtypes = [P]
         for f in ("la_prefill", "la_prefill_varlen", "la_prefill_with_state",
                   "la_prefill_varlen_with_state", "la_mixed_step", "la_output_norm_gate",
                   "la_state_prefix", "la_prefill_state",
                   "la_decode", "la_backward",
                   "la_read_device_status", "la_set_tuning", "la_get_tuning",
-                  "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection"):
+                  "la_last_launch_count", "la_prefill_noalloc", "la_set_fault_injection",
+                  "la_noalloc_device_status"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -200,6 +202,11 @@ def la_prefill_noalloc(q, k, v, slopes, o, state_out, stream=None):
     _check("la_prefill_noalloc", lib().la_prefill_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(slopes), _ptr(o), _ptr(state_out), B, H, N, d,
         _dt(q), _dt(o), _stream(stream)))
+
+
+def la_noalloc_device_status(stream=None) -> int:
+    """Device-side status of the last la_prefill_noalloc on the current device."""
+    return int(lib().la_noalloc_device_status(_stream(stream)))
 
 
 def la_read_device_status(ws, stream=None) -> int:

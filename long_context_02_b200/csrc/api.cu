@@ -138,6 +138,8 @@ int prefill_varlen(const int* cu_seqlens, int num_seqs, const void* q, const voi
 {
     g_launches = 0;
     if (num_seqs < 0 || H <= 0 || total < 0) return LA_ERR_INVALID_ARG;
+    // Tokens without sequences would be left unwritten: the arguments disagree.
+    if (num_seqs == 0 && total > 0) return LA_ERR_INVALID_ARG;
     if (check_sizes(num_seqs, H, total) != LA_OK) return LA_ERR_UNSUPPORTED;
     int st = check_d(d);
     if (st != LA_OK) return st;
@@ -248,6 +250,8 @@ LA_API int la_mixed_step(const int* cu_seqlens, int num_seqs, const void* q, con
 {
     g_launches = 0;
     if (num_seqs < 0 || H <= 0 || total < 0) return LA_ERR_INVALID_ARG;
+    // Tokens without sequences would be left unwritten: the arguments disagree.
+    if (num_seqs == 0 && total > 0) return LA_ERR_INVALID_ARG;
     if (check_sizes(num_seqs, H, total) != LA_OK) return LA_ERR_UNSUPPORTED;
     int st = check_d(d);
     if (st != LA_OK) return st;

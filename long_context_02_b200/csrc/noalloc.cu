@@ -72,3 +72,19 @@ extern "C" LA_API int la_prefill_noalloc(const void* q, const void* k, const voi
     return la_prefill(q, k, v, slopes, o, state_out, B, H, N, d, in_t, out_t, scratch,
                       kScratchBytes, stream);
 }
+
+extern "C" LA_API int la_noalloc_device_status(la_stream_t stream)
+{
+    // The status word sits at the start of the built-in scratch, where
+    // la_prefill writes device-side errors (a bounded wait that gave up). It is
+    // read into a host int with a plain copy: nothing is allocated here either.
+    int status = LA_OK;
+    void* scratch = scratch_on_current_device(&status);
+    if (scratch == nullptr) return status;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return LA_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LA_ERR_CUDA;
+    return word;
+}

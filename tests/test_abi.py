@@ -103,6 +103,13 @@ def test_varlen_argument_errors(lib):
                                  None) == B.LA_ERR_INVALID_ARG
     assert lib.la_prefill_varlen(P(18), 2, x, x, x, x, x, None, 4, 100, 128, 0, 0, x, 1 << 30,
                                  None) == B.LA_ERR_INVALID_ARG
+    # tokens but no sequences: the arguments disagree (O would be left unwritten)
+    assert lib.la_prefill_varlen(x, 0, x, x, x, x, x, None, 4, 100, 128, 0, 0, x, 1 << 30,
+                                 None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_prefill_varlen_with_state(x, 0, x, x, x, x, None, x, None, 4, 100, 128, 0, 0,
+                                            x, 1 << 30, None) == B.LA_ERR_INVALID_ARG
+    assert lib.la_mixed_step(x, 0, x, x, x, x, None, x, 4, 100, 128, 0, 0, x, 1 << 30, None,
+                             None) == B.LA_ERR_INVALID_ARG
 
 
 def test_with_state_argument_errors(lib):
