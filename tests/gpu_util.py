@@ -48,3 +48,18 @@ def assert_close_bf16_out(got, ref, tol, what=""):
     bound = tol * rms(ref) + BF16_ULP * np.abs(ref)
     bad = np.abs(got - ref) > bound
     assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond tol*rms + 2^-8|ref|"
+
+
+def assert_close_heads(got, ref, tol, heads, what="", axis=0):
+    """The tolerance over the compared tensor, and again inside each head:
+    max |err| <= tol * rms(ref of that head), so that a fast-decay head with a
+    small output cannot hide its errors under a slow head's larger rms.
+    `axis` is the head axis of `got` and `ref`; `heads` names its entries."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    worst = assert_close(got, ref, tol, what)
+    for i, h in enumerate(heads):
+        e = assert_close(np.take(got, i, axis=axis), np.take(ref, i, axis=axis), tol,
+                         f"{what}, head {h} alone")
+        worst = max(worst, e)
+    return worst
