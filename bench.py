@@ -296,7 +296,7 @@ def run_ours(args):
                "schedule": f"{groups} head groups, copy-in / prefill / copy-out on 3 streams"}
         del hq, hk, hv, ho, hst
 
-    secondary = {} if args.no_secondary else run_secondary(args, L, inputs, dev, world, pk)
+    secondary = {} if args.no_secondary else run_secondary(args, L, inputs, dev, world, pk, rank)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -369,7 +369,38 @@ def bench_mixed(L, inputs, dev, world, steps):
     return res
 
 
-def run_secondary(args, L, inputs, dev, world, pk):
+def bench_sp(L, inputs, dev, world, rank, steps):
+    """One MiniMax-shaped sequence (B=1, H=64, N=32768, d=128, bf16) cut into
+    `world` consecutive chunks, one per rank: every rank runs sp.sp_prefill on
+    its chunk with the NCCL all-gather of the local states (4 MiB per rank)
+    inside the timed region. The rate is the whole sequence's FLOPs over the
+    slowest rank's time (strong scaling of one sequence)."""
+    from long_context_02_b200 import sp
+    n = N_ // world
+    q, k, v, s = inputs.prefill_inputs(1, H_, N_, D_, torch.bfloat16, dev, seed=19)
+    qc, kc, vc = (t[:, :, rank * n:(rank + 1) * n].contiguous() for t in (q, k, v))
+    del q, k, v
+    o = torch.empty_like(qc)
+    st = torch.empty((1, H_, D_, D_), dtype=torch.float32, device=dev)
+    ws = L.workspace(L.LA_OP_PREFILL, 1, H_, n, D_, 0, torch.bfloat16, dev)
+    gather = sp.nccl_gather()
+    fn = lambda: sp.sp_prefill(qc, kc, vc, s, [n] * world, rank, o, st, gather, ws)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    assert L.la_read_device_status(ws) == L.LA_OK
+    ms = timed(fn, steps, world)
+    F = prefill_flops(1, H_, N_)
+    res = {"workload": f"sequence-parallel prefill of one B=1 H=64 N={N_} d=128 bf16 sequence "
+                       f"over {world} ranks ({n}-token chunks); local state, NCCL all-gather "
+                       "of the local states, prefix, prefill from it: all timed",
+           "ms": round(ms, 4), "TFLOP/s": round(F / (ms * 1e-3) / 1e12, 2),
+           "tokens_per_s": round(N_ / (ms * 1e-3), 1), "scaling": "strong"}
+    del qc, kc, vc, o, st, ws
+    return res
+
+
+def run_secondary(args, L, inputs, dev, world, pk, rank=0):
     out = {}
     steps = max(3, min(args.steps, 50))
     # decode: batch 256, H=64, d=128, fp32 state [256,64,128,128] ~ N(0, 0.01)
@@ -454,6 +485,8 @@ def run_secondary(args, L, inputs, dev, world, pk):
                     "prefill from that state; all-gather not included)",
         "ms": round(ms, 4)}
     del q, k, v, o, st, states, ws
+    if world > 1:
+        out["sp"] = bench_sp(L, inputs, dev, world, rank, steps)
     # output normalization and gate on the prefill's output (bf16 O, gate and Y)
     o = torch.randn((1, 64, 32768, 128), device=dev).to(torch.bfloat16)
     g = torch.randn((1, 32768, 64 * 128), device=dev).to(torch.bfloat16)
@@ -538,7 +571,41 @@ def cpu_baseline(n_heads=64, threads=None, seed=0):
     return {"value": round(F / dt / 1e12, 6), "unit": "TFLOP/s", "cores": th, "kind": "oracle",
             "sample": f"fp64 token recurrence on {n_heads} of 64 heads x {N_} tokens, d=128 "
                       f"({dt:.1f} s)",
-            "tokens_per_s": round(N_ * n_heads / 64 / dt, 1)}
+            "tokens_per_s": round(N_ * n_heads / 64 / dt, 1),
+            "quadratic_form": cpu_quadratic_sample(qn, kn, vn, orc, th)}
+
+
+def cpu_quadratic_sample(qn, kn, vn, orc, threads, n_heads=8, stride=16):
+    """The oracle's quadratic form (the operator's definition, O(N^2 d) per head)
+    timed on a labelled sample of the headline workload and extrapolated to the
+    whole of it. Sample: rows i = stride-1, 2*stride-1, ..., N-1 of n_heads heads
+    (data of the first heads, decays of heads spread over 0..63). Row i costs
+    (i+1) terms, so the whole workload's time is the sample's time times
+    64 * N(N+1)/2 over the sample's sum of (i+1)."""
+    import numpy as np
+
+    import oracle
+    from long_context_02_b200 import inputs
+    lam_all = oracle.lambdas_from_slopes(inputs.slopes(H_).numpy())
+    heads = [round(x) for x in np.linspace(0, H_ - 1, n_heads)]
+    rows = np.arange(stride - 1, N_, stride, dtype=np.int64)
+    n_heads = min(n_heads, qn.shape[1])
+    t0 = time.perf_counter()
+    for i in range(n_heads):
+        orc.forward_rows(qn[0, i], kn[0, i], vn[0, i], lam_all[heads[i]], rows)
+    dt = time.perf_counter() - t0
+    terms_sample = n_heads * float(np.sum(rows + 1))
+    terms_full = H_ * N_ * (N_ + 1) / 2.0
+    t_full = dt * terms_full / terms_sample
+    F = prefill_flops(1, H_, N_)
+    return {"value": round(F / t_full / 1e12, 8), "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle (quadratic form)",
+            "sample": f"quadratic-form rows {stride - 1}, {2 * stride - 1}, ..., {N_ - 1} "
+                      f"({len(rows)} rows) of {n_heads} heads (decays of heads {heads}), "
+                      f"{dt:.1f} s",
+            "extrapolated_s": round(t_full, 1),
+            "extrapolation": "t_full = t_sample * (64 * N(N+1)/2) / (sum over sampled "
+                             "(head, row i) of (i+1))"}
 
 
 def run_reference(args):

@@ -39,6 +39,23 @@ def nccl_gather(group=None) -> Callable[[torch.Tensor], torch.Tensor]:
     return gather
 
 
+def host_gather(group=None) -> Callable[[torch.Tensor], torch.Tensor]:
+    """All-gather of one tensor per rank staged through host memory, for process
+    groups whose backend moves CPU tensors only (gloo): the local state is copied
+    to the host, gathered, and the [world, *shape] result copied back to the
+    tensor's device."""
+    import torch.distributed as dist
+
+    def gather(x: torch.Tensor) -> torch.Tensor:
+        world = dist.get_world_size(group)
+        xc = x.detach().to("cpu").contiguous()
+        parts = [torch.empty_like(xc) for _ in range(world)]
+        dist.all_gather(parts, xc, group=group)
+        return torch.stack(parts).to(x.device)
+
+    return gather
+
+
 def local_state(k, v, slopes, ws, stream=None) -> torch.Tensor:
     """Step 1: the state of this rank's chunk alone, [B,H,d,d] fp32."""
     B, H, _, d = k.shape

@@ -27,3 +27,24 @@ def test_profiled_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     prof.write_text("kernel_source_sha256_16: 0000000000000000\ndram_bytes_per_full_launch: 1\n")
     assert bench.profiled_traffic() is None
 
+
+
+def test_quadratic_form_sample_extrapolates_by_the_row_costs():
+    """The CPU baseline's quadratic-form leg: a sample of rows, scaled to the
+    whole workload by the number of (i+1) terms (here one head, rows 4095,
+    8191, ..., 32767)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from long_context_02_b200 import inputs
+    q, k, v, _ = inputs.prefill_inputs(1, 1, bench.N_, bench.D_, torch.bfloat16, "cpu", seed=0)
+    f = lambda t: t.to(torch.float64).numpy()
+    r = bench.cpu_quadratic_sample(f(q), f(k), f(v), oracle.default(), 1, n_heads=1,
+                                   stride=4096)
+    rows = np.arange(4095, bench.N_, 4096)
+    ratio = 64 * bench.N_ * (bench.N_ + 1) / 2 / float(np.sum(rows + 1))
+    t_sample = r["extrapolated_s"] / ratio
+    assert r["value"] > 0 and r["extrapolated_s"] > 0
+    want = bench.prefill_flops(1, 64, bench.N_) / (t_sample * ratio) / 1e12
+    assert abs(r["value"] - want) <= 1e-3 * want  # both figures are rounded in the report

@@ -15,6 +15,7 @@ import socket
 import subprocess
 import sys
 
+import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -80,7 +81,7 @@ def test_reference_arm_line(tmp_path):
     assert line["e2e"]["h2d_bytes_per_step"] == 0
 
 
-def _sp_rank_main(rank, world, port, out):
+def _sp_rank_main(rank, world, port, out, which="nccl_gather"):
     import datetime
 
     import numpy as np
@@ -100,7 +101,7 @@ def _sp_rank_main(rank, world, port, out):
     a = sum(lens[:rank])
     b = a + lens[rank]
     _, s_loc = oracle.forward(q[:, :, a:b], k[:, :, a:b], v[:, :, a:b], lam)
-    states = sp.nccl_gather()(torch.from_numpy(s_loc))   # the exchange under test
+    states = getattr(sp, which)()(torch.from_numpy(s_loc))   # the exchange under test
     s_in = oracle.state_prefix(states.numpy(), lam, lens, rank)
     _, want = oracle.forward(q[:, :, :a], k[:, :, :a], v[:, :, :a], lam)
     ok = tuple(states.shape) == (world, B, H, d, d) and np.allclose(s_in, want, rtol=1e-12,
@@ -110,11 +111,12 @@ def _sp_rank_main(rank, world, port, out):
     dist.destroy_process_group()
 
 
-def test_sequence_parallel_exchange_two_ranks():
+@pytest.mark.parametrize("which", ["nccl_gather", "host_gather"])
+def test_sequence_parallel_exchange_two_ranks(which):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_sp_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_sp_rank_main, args=(r, 2, port, q, which)) for r in range(2)]
     for p in procs:
         p.start()
     res = sorted(q.get(timeout=120) for _ in range(2))
