@@ -30,8 +30,9 @@
 //     MMA1  SP  = Q K^T                    (fp32, TMEM)
 //     E_P   P   = SP * lam^(i-j) [j<=i]     written back into TMEM as bf16 hi + lo
 //     MMA2  OI  = P_hi V + P_lo V           (A operand from TMEM)
-//     MMA3  OE  = Q S_hi + Q S_lo           (bf16 hi + lo copies of the fp32 state)
-//     E_O   O   = OI + lam^(i+1) OE  -> global (bf16 or fp32)
+//     MMA3  [OE_hi | OE_lo] = Q [S_hi | S_lo]   (bf16 hi + lo copies of the fp32 state,
+//                                              side by side: one N = 128 MMA per k-step)
+//     E_O   O   = OI + lam^(i+1) (OE_hi + OE_lo)  -> global (bf16 or fp32)
 //     E_V   Vd  = lam^(L-1-j) v_j           (bf16 hi + lo, shared memory)
 //     MMA4  DS  = K^T Vd_hi + K^T Vd_lo
 //     E_S   S   = lam^L S + DS              (fp32 in registers; hi + lo copies for MMA3)
@@ -48,7 +49,15 @@
 // Warp roles (16 warps, 4 warpgroups): warp 0 TMA producer, warp 1 MMA issuer
 // (also owns TMEM); warps 4-7 "P" (E_P); warps 8-11 "VO" (E_V, E_O); warps
 // 12-15 "S" (E_S and the scan; the fp32 state lives in their registers, one
-// key row a per thread). TMEM: 512 columns = SP[2] | OI | DS | OE[2].
+// key row a per thread). TMEM: 512 columns = SP[2] | OI | DS | OE, with OE
+// holding [OE_hi | OE_lo].
+//
+// Shared memory is the resource every step competes for: the MMAs' operand
+// reads (both operands of the smem-operand forms), the TMA writes and the
+// epilogues' loads and stores all share its 128 bytes per clock, and an
+// mbarrier probe queues behind them. Hence MMA3 reads Q once for both state
+// copies (N = 128), and the MMA warp probes every barrier a group needs at
+// once (wait_multi), so that MMA4 and MMA3 issue back to back.
 // Shared memory: two slots each for Q, K (128 x 128) and V (128 x 64), the
 // decayed values (hi, lo) and the state copies (hi, lo), all in the 128-byte
 // swizzled layout TMA writes.
@@ -76,6 +85,7 @@ constexpr int NUM_THREADS = 512;                 // 4 warpgroups
 // launched at 65536 / 512 = 128 per thread. 128 * (104 + 120 + 128 + 152) =
 // 64512 <= 65536.
 constexpr int REGS_CTRL = 104, REGS_P = 120, REGS_VO = 128, REGS_S = 152;
+static_assert(128 * (REGS_CTRL + REGS_P + REGS_VO + REGS_S) <= 65536, "register split");
 constexpr uint32_t BOX_BYTES = 128 * 64 * 2;     // one TMA box: 128 rows x 64 bf16
 constexpr uint32_t TILE_BYTES = 2 * BOX_BYTES;   // 128 x 128 bf16
 // Tile region (1024-aligned).
@@ -88,7 +98,7 @@ constexpr uint32_t OFF_SH = OFF_VL + BOX_BYTES;        // state copy, hi
 constexpr uint32_t OFF_SL = OFF_SH + BOX_BYTES;        // state copy, lo
 constexpr uint32_t SMEM_TILES = OFF_SL + BOX_BYTES;    // 224 KB
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_SP = 0, COL_OI = 256, COL_DS = 320, COL_OE = 384;
+constexpr uint32_t COL_SP = 0, COL_OI = 256, COL_DS = 320, COL_OE = 384;  // OE: 128 columns
 constexpr unsigned long long WAIT_LIMIT_NS = 4000000000ull;
 constexpr unsigned long long FLAG_LIMIT_NS = 2000000000ull;
 constexpr unsigned long long DRAIN_LIMIT_NS = 200000000ull;
@@ -105,7 +115,8 @@ enum {
     B_VH_FREE, B_VH_READY,           // decayed values: MMA4 done / E_V done
     B_DS_FULL, B_DS_EMPTY,           // DS: MMA4 done / E_S read it
     B_S_FREE, B_S_READY,             // state copy: MMA3 done / E_S wrote it
-    B_O_FULL, B_O_EMPTY,             // OI, OE: MMA2 done / E_O read them
+    B_O_FULL, B_O_EMPTY,             // OI: MMA2 done / E_O read it
+    B_OE_FREE,                       // OE: E_O read it (MMA3 may write it)
     B_ITEM_FULL0, B_ITEM_FULL1, B_ITEM_EMPTY0, B_ITEM_EMPTY1,
     B_FIN, B_P_SYNC, B_S_SYNC,
     NUM_BARS
@@ -122,7 +133,7 @@ constexpr uint32_t idesc(uint32_t n, uint32_t a_mn_major, uint32_t b_mn_major)
 }
 constexpr uint32_t IDESC_QK = idesc(128, 0, 0);  // Q K^T: both K-major
 constexpr uint32_t IDESC_PV = idesc(64, 0, 1);   // P (TMEM) V: V MN-major
-constexpr uint32_t IDESC_QS = idesc(64, 0, 1);   // Q S: S rows = key dim, MN-major
+constexpr uint32_t IDESC_QS = idesc(128, 0, 1);  // Q [S_hi | S_lo]: rows = key dim, MN-major
 constexpr uint32_t IDESC_KV = idesc(64, 1, 1);   // K^T Vd: both MN-major
 
 struct Params {
@@ -243,6 +254,19 @@ __device__ __forceinline__ bool wait_warp(uint64_t* b, uint32_t parity, volatile
     return __all_sync(0xffffffffu, ok);
 }
 
+// Warp-uniform bounded wait on up to three barriers at once: lane i probes
+// barrier i (lanes past n probe barrier 0), so the probes go out together
+// instead of one round trip each.
+__device__ __forceinline__ bool wait_multi(int n, uint64_t* b0, uint32_t p0, uint64_t* b1,
+                                           uint32_t p1, uint64_t* b2, uint32_t p2, int lane,
+                                           volatile int* abort, WsHeader* hdr)
+{
+    uint64_t* b = (lane == 1 && n > 1) ? b1 : (lane == 2 && n > 2) ? b2 : b0;
+    const uint32_t par = (lane == 1 && n > 1) ? p1 : (lane == 2 && n > 2) ? p2 : p0;
+    if (__all_sync(0xffffffffu, mbar_try_wait(b, par))) return true;
+    return __all_sync(0xffffffffu, mbar_wait_slow(b, par, abort, hdr, WAIT_LIMIT_NS));
+}
+
 // Bounded barrier over one 128-thread group (an mbarrier of count 128).
 __device__ __forceinline__ bool group_sync(uint64_t* b, uint32_t& n, volatile int* abort,
                                            WsHeader* hdr)
@@ -347,6 +371,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
 {
     asm volatile(
@@ -394,6 +430,12 @@ __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
 {
     uint64_t r;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
 __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b)
@@ -634,7 +676,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
     const uint64_t dkm0 = sdesc(smem_u32(sm.k(0)), BOX_BYTES, 1024u);
     const uint64_t dv0 = sdesc(smem_u32(sm.v(0)), 16u, 1024u);
     const uint64_t dvh = sdesc(smem_u32(sm.vh()), 16u, 1024u);
-    const uint64_t dsh = sdesc(smem_u32(sm.sh()), 16u, 1024u);
+    const uint64_t dsh = sdesc(smem_u32(sm.sh()), BOX_BYTES, 1024u);  // [S_hi | S_lo], N = 128
     constexpr uint64_t TILE16 = TILE_BYTES >> 4, BOX16 = BOX_BYTES >> 4;
     // nq, nkv: Q / K-V loads consumed; g: phase-C blocks; n_ds: DS productions;
     // n_vh: decayed-value tiles; n_s: state copies.
@@ -661,8 +703,9 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
     // SP[g & 1] = Q K^T for phase-C block g (Q slot nq, K slot nkv).
     auto mma1 = [&](uint32_t gg, uint32_t q_use, uint32_t kv_use) -> bool {
         const int sq = q_use & 1, sk = kv_use & 1;
-        if (!wait_warp(&bars[B_QF0 + sq], (q_use >> 1) & 1, sm.abort, p.hdr)) return false;
-        if (!wait_warp(&bars[B_KF0 + sk], (kv_use >> 1) & 1, sm.abort, p.hdr)) return false;
+        if (!wait_multi(2, &bars[B_QF0 + sq], (q_use >> 1) & 1, &bars[B_KF0 + sk],
+                        (kv_use >> 1) & 1, nullptr, 0, lane, sm.abort, p.hdr))
+            return false;
         tc_fence_after();
         const uint64_t a = dq0 + (uint64_t)sq * TILE16, b = dk0 + (uint64_t)sk * TILE16;
         const uint32_t d = tmem + COL_SP + 128u * (gg & 1);
@@ -717,8 +760,11 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             const int sq = (q0 + kb) & 1, skv = (kv0 + kb) & 1;
             // MMA4: this block's DS, once E_V has decayed its values and E_S
             // has read the previous DS.
-            ok = wait_warp(&bars[B_VH_READY], n_vh & 1, sm.abort, p.hdr) &&
-                 wait_warp(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr);
+            // One probe for everything MMA4 and MMA3 need: the decayed values,
+            // DS read by E_S, and the state copy (which E_S writes after reading
+            // the previous DS), so that the two groups issue back to back.
+            ok = wait_multi(3, &bars[B_VH_READY], n_vh & 1, &bars[B_DS_EMPTY], (n_ds & 1) ^ 1,
+                            &bars[B_S_READY], n_s & 1, lane, sm.abort, p.hdr);
             if (!ok) break;
             ++n_vh;
             tc_fence_after();
@@ -730,21 +776,19 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             }
             __syncwarp();
             ++n_ds;
-            // MMA3: OE[g & 1] = Q S_in (hi and lo), once E_S has written the copy.
-            ok = wait_warp(&bars[B_S_READY], n_s & 1, sm.abort, p.hdr);
-            if (!ok) break;
+            // MMA3: [OE_hi | OE_lo] = Q [S_hi | S_lo]; the copy was waited for above,
+            // OE must have been read by E_O of the previous block.
             ++n_s;
+            ok = wait_warp(&bars[B_OE_FREE], (gg & 1) ^ 1, sm.abort, p.hdr);
+            if (!ok) break;
             tc_fence_after();
             {
                 const uint64_t a = dq0 + (uint64_t)sq * TILE16;
-                const uint32_t d = tmem + COL_OE + (uint32_t)DV * (gg & 1);
+                const uint32_t d = tmem + COL_OE;
                 if (elect_one()) {
 #pragma unroll
-                    for (int part = 0; part < 2; ++part)
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks)
-                            mma_ss(d, a + koff_k(ks), dsh + part * BOX16 + koff_mn(ks), IDESC_QS,
-                                   (part || ks) ? 1u : 0u);
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_ss(d, a + koff_k(ks), dsh + koff_mn(ks), IDESC_QS, ks ? 1u : 0u);
                     mma_commit(&bars[B_S_FREE]);
                     mma_commit(&bars[B_QE0 + sq]);
                 }
@@ -754,8 +798,8 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             if (kb + 1 < nb && !(ok = mma1(gg + 1, q0 + kb + 1, kv0 + kb + 1))) break;
             // MMA2: OI = P V (P hi and lo from TMEM), once E_P is done and
             // E_O has read the previous OI.
-            ok = wait_warp(&bars[B_P_READY0 + (gg & 1)], (gg >> 1) & 1, sm.abort, p.hdr) &&
-                 wait_warp(&bars[B_O_EMPTY], (gg & 1) ^ 1, sm.abort, p.hdr);
+            ok = wait_multi(2, &bars[B_P_READY0 + (gg & 1)], (gg >> 1) & 1, &bars[B_O_EMPTY],
+                            (gg & 1) ^ 1, nullptr, 0, lane, sm.abort, p.hdr);
             if (!ok) break;
             tc_fence_after();
             {
@@ -916,7 +960,9 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         const float f = row < L ? expf(-slope * (float)m) : 0.f;
         const uint64_t ff = f2(f, f);
         const uint8_t* src = sm.v(s);
-#pragma unroll 1
+        // Two 16-byte chunks in flight: E_V sits between this block's MMA4 and
+        // the next one, and its latency, not its instruction count, is what counts.
+#pragma unroll 2
         for (int c = 0; c < 8; ++c) {
             const uint4 u = *reinterpret_cast<const uint4*>(src + swz(row, c));
             uint4 h, l;
@@ -966,27 +1012,33 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
             const bool store = row < L;
             const long long orow = it.out_row0 + t0 + row;
 #pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                uint32_t ri[32], re[32];
-                tmem_ld32(lane_addr + COL_OI + 32 * h, ri);
-                tmem_ld32(lane_addr + COL_OE + (uint32_t)DV * (g & 1) + 32 * h, re);
+            for (int c = 0; c < 4; ++c) {
+                uint32_t ri[16], rh[16], rl[16];
+                tmem_ld16(lane_addr + COL_OI + 16 * c, ri);
+                tmem_ld16(lane_addr + COL_OE + 16 * c, rh);
+                tmem_ld16(lane_addr + COL_OE + DV + 16 * c, rl);
                 tmem_wait_ld();
-                uint64_t ov[16];
+                if (c == 3) {
+                    tc_fence_before();
+                    mbar_arrive(&bars[B_OE_FREE]);
+                }
+                uint64_t ov[8];
 #pragma unroll
-                for (int x = 0; x < 16; ++x)
-                    ov[x] = fma2(rc2, f2u(re[2 * x], re[2 * x + 1]), f2u(ri[2 * x], ri[2 * x + 1]));
+                for (int x = 0; x < 8; ++x)
+                    ov[x] = fma2(rc2, add2(f2u(rh[2 * x], rh[2 * x + 1]), f2u(rl[2 * x], rl[2 * x + 1])),
+                                 f2u(ri[2 * x], ri[2 * x + 1]));
                 if (store) {
-                    const size_t off = (size_t)orow * D + DV * it.half + 32 * h;
+                    const size_t off = (size_t)orow * D + DV * it.half + 16 * c;
                     if (OUT_F32) {
                         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + off);
 #pragma unroll
-                        for (int x = 0; x < 8; ++x)
+                        for (int x = 0; x < 4; ++x)
                             dst[x] = make_float4(f2x(ov[2 * x]), f2y(ov[2 * x]), f2x(ov[2 * x + 1]),
                                                  f2y(ov[2 * x + 1]));
                     } else {
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + off);
 #pragma unroll
-                        for (int x = 0; x < 4; ++x)
+                        for (int x = 0; x < 2; ++x)
                             dst[x] = make_uint4(pack_bf16x2(f2x(ov[4 * x + 0]), f2y(ov[4 * x + 0])),
                                                 pack_bf16x2(f2x(ov[4 * x + 1]), f2y(ov[4 * x + 1])),
                                                 pack_bf16x2(f2x(ov[4 * x + 2]), f2y(ov[4 * x + 2])),
@@ -1162,8 +1214,8 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
 // Small shared state at the start of the dynamic region; the 1024-aligned
 // tile region follows (SMEM_BYTES reserves the worst-case alignment gap).
 constexpr uint32_t SM_BARS = 0;                       // NUM_BARS x 8 B
-constexpr uint32_t SM_RING = 256;                     // 2 x Item
-constexpr uint32_t SM_PW = 384;                       // (C + 1) floats
+constexpr uint32_t SM_RING = 320;                     // 2 x Item
+constexpr uint32_t SM_PW = 448;                       // (C + 1) floats
 constexpr uint32_t SM_TMEM = SM_PW + 4 * (C + 4);     // u32
 constexpr uint32_t SM_ABORT = SM_TMEM + 4;            // int
 constexpr uint32_t SM_SMALL = SM_ABORT + 4;
@@ -1195,7 +1247,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int i = 0; i < NUM_BARS; ++i) {
             uint32_t count = 1;  // TMA expect_tx arrivals, MMA commits, single threads
             if (i == B_P_READY0 || i == B_P_READY1 || i == B_VH_READY || i == B_DS_EMPTY ||
-                i == B_S_READY || i == B_O_EMPTY || i == B_P_SYNC || i == B_S_SYNC)
+                i == B_S_READY || i == B_O_EMPTY || i == B_OE_FREE || i == B_P_SYNC ||
+                i == B_S_SYNC)
                 count = 128;
             if (i == B_ITEM_EMPTY0 || i == B_ITEM_EMPTY1) count = 1 + 12;  // MMA lane + 12 group warps
             mbar_init(&bars[i], count);
@@ -1516,8 +1569,14 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     const long long max_items = 2 * w.max_items;
     const int grid = (int)std::min<long long>(num_sms(), std::max<long long>(1, max_items));
     auto launch = [&](auto kern) -> cudaError_t {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_BYTES);
+        // The warpgroups' setmaxnreg split assumes the CTA launches with 128
+        // registers per thread; with fewer, the S group's increase would wait forever.
+        cudaFuncAttributes fa{};
+        cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != 65536 / NUM_THREADS) return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
         kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
         count_launch();
