@@ -94,35 +94,101 @@ def profiled_traffic():
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples of SM clocks and throttle reasons during the timed region."""
+    """SM clock, power and clock-event reasons while the timed loop runs.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Sampled through NVML (the library nvidia-smi reports from) every ~1 ms in a
+    background thread; only samples inside the window that timed() marks with
+    begin()/end() count as "under load". The timed region is short (20 prefill
+    steps take ~12 ms), so a sampler at nvidia-smi's 50 ms period would mostly
+    see the idle GPU around it. Falls back to nvidia-smi samples when NVML is
+    unavailable."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
 
     def __init__(self, device):
+        self.samples = []
+        self.window = None
+        self.thread = None
         self.proc = None
-        self.path = None
+        self.nvml = None
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:
             self.gpu = str(device)
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(self.gpu)
+            self.nvml = pynvml
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        n = self.nvml
+        max_mhz = n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM)
+        while not self.stop_flag:
+            try:
+                mhz = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+                reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                watts = n.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                self.samples.append((time.perf_counter(), float(mhz), float(max_mhz), int(reasons),
+                                     watts))
+            except Exception:
+                pass
+            time.sleep(0.001)
 
     def start(self):
+        import threading
+        self.samples, self.window = [], None
+        if self.nvml is not None:
+            self.stop_flag = False
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+            time.sleep(0.01)
+            return
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.out = open(self.path, "w")
+            fields = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                      "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                      "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={fields}",
                  "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.out, stderr=subprocess.DEVNULL)
             time.sleep(0.3)
         except Exception:
             self.proc = None
 
+    def begin(self):
+        self.window = [time.perf_counter(), None]
+
+    def end(self):
+        if self.window is not None and self.window[1] is None:
+            self.window[1] = time.perf_counter()
+
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            rows = self.samples
+            if self.window and self.window[1] is not None:
+                inside = [r for r in rows if self.window[0] <= r[0] <= self.window[1]]
+            else:
+                inside = []
+            use = inside or rows
+            if not use:
+                return None
+            reasons = sorted({name for r in use for name, bit in self.REASONS if r[3] & bit})
+            return {"sm_mhz": statistics.median(r[1] for r in use),
+                    "sm_mhz_min": min(r[1] for r in use),
+                    "sm_max_mhz": max(r[2] for r in use), "reasons": reasons,
+                    "power_w_max": round(max(r[4] for r in use), 1),
+                    "samples": len(use), "under_load": bool(inside), "source": "nvml, 1 ms"}
         if self.proc is None:
             return None
         time.sleep(0.1)
@@ -151,7 +217,7 @@ class ClockSampler:
                           if r[i].lower() in ("active", "1", "yes")})
         return {"sm_mhz": statistics.median(r[0] for r in rows),
                 "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "under_load": False, "source": "nvidia-smi, 50 ms"}
 
 
 # ---------------------------------------------------------------- distributed
@@ -195,17 +261,22 @@ def whole_job_rate(units_per_rank, local_ms, world):
     return ms, world * units_per_rank / (ms * 1e-3)
 
 
-def timed(fn, steps, world, stream=None):
-    """Device time of `steps` calls of fn (ms per step), max over ranks."""
+def timed(fn, steps, world, stream=None, sampler=None):
+    """Device time of `steps` calls of fn (ms per step), max over ranks. A clock
+    sampler, if given, counts only the samples taken while the loop runs."""
     stream = stream or torch.cuda.current_stream()
     barrier(world)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    if sampler is not None:
+        sampler.begin()
     for _ in range(steps):
         fn()
     b.record(stream)
     torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.end()
     barrier(world)
     return max_over_ranks(a.elapsed_time(b) / steps, world)
 
@@ -236,7 +307,7 @@ def run_ours(args):
     launches_per_step = L.la_last_launch_count()
     sampler = ClockSampler(dev)
     sampler.start()
-    ms = timed(step, args.steps, world)
+    ms = timed(step, args.steps, world, sampler=sampler)
     clocks = sampler.stop()
     assert L.la_read_device_status(ws) == L.LA_OK
 

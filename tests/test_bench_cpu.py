@@ -48,3 +48,23 @@ def test_quadratic_form_sample_extrapolates_by_the_row_costs():
     assert r["value"] > 0 and r["extrapolated_s"] > 0
     want = bench.prefill_flops(1, 64, bench.N_) / (t_sample * ratio) / 1e12
     assert abs(r["value"] - want) <= 1e-3 * want  # both figures are rounded in the report
+
+
+def test_clock_sampler_counts_only_samples_inside_the_timed_loop():
+    """bench.ClockSampler reports the clocks of the samples taken while the
+    timed loop ran (the window timed() marks), not the idle GPU around it."""
+    import threading
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples = [(0.0, 1965.0, 1965.0, 0x1, 200.0),     # idle, before
+                 (1.0, 1600.0, 1965.0, 0x4, 990.0),     # under load, power cap
+                 (1.5, 1650.0, 1965.0, 0x4, 1001.0),
+                 (3.0, 1965.0, 1965.0, 0x1, 250.0)]     # idle, after
+    s.window = [0.9, 2.0]
+    s.thread = threading.Thread(target=lambda: None)
+    s.thread.start()
+    s.stop_flag = False
+    s.proc = None
+    r = s.stop()
+    assert r["under_load"] and r["samples"] == 2
+    assert r["sm_mhz"] == 1625.0 and r["sm_mhz_min"] == 1600.0
+    assert r["reasons"] == ["sw_power_cap"] and r["power_w_max"] == 1001.0
