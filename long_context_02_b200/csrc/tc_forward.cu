@@ -762,9 +762,14 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             // has read the previous DS.
             // One probe for everything MMA4 and MMA3 need: the decayed values,
             // DS read by E_S, and the state copy (which E_S writes after reading
-            // the previous DS), so that the two groups issue back to back.
-            ok = wait_multi(3, &bars[B_VH_READY], n_vh & 1, &bars[B_DS_EMPTY], (n_ds & 1) ^ 1,
-                            &bars[B_S_READY], n_s & 1, lane, sm.abort, p.hdr);
+            // the previous DS), so that the two groups issue back to back. The
+            // first block's copy is made from the scan's prefix or the caller's
+            // state, which E_S reads from global memory: MMA4 does not wait for it.
+            ok = kb > 0 ? wait_multi(3, &bars[B_VH_READY], n_vh & 1, &bars[B_DS_EMPTY],
+                                     (n_ds & 1) ^ 1, &bars[B_S_READY], n_s & 1, lane, sm.abort,
+                                     p.hdr)
+                        : wait_multi(2, &bars[B_VH_READY], n_vh & 1, &bars[B_DS_EMPTY],
+                                     (n_ds & 1) ^ 1, nullptr, 0, lane, sm.abort, p.hdr);
             if (!ok) break;
             ++n_vh;
             tc_fence_after();
@@ -776,10 +781,12 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             }
             __syncwarp();
             ++n_ds;
-            // MMA3: [OE_hi | OE_lo] = Q [S_hi | S_lo]; the copy was waited for above,
-            // OE must have been read by E_O of the previous block.
+            // MMA3: [OE_hi | OE_lo] = Q [S_hi | S_lo], once E_O of the previous block
+            // has read OE (and, for the first block, E_S has written the copy).
+            ok = kb > 0 ? wait_warp(&bars[B_OE_FREE], (gg & 1) ^ 1, sm.abort, p.hdr)
+                        : wait_multi(2, &bars[B_OE_FREE], (gg & 1) ^ 1, &bars[B_S_READY],
+                                     n_s & 1, nullptr, 0, lane, sm.abort, p.hdr);
             ++n_s;
-            ok = wait_warp(&bars[B_OE_FREE], (gg & 1) ^ 1, sm.abort, p.hdr);
             if (!ok) break;
             tc_fence_after();
             {
