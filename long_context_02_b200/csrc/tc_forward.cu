@@ -113,6 +113,7 @@ enum {
     B_SP_FULL0, B_SP_FULL1,          // MMA1 done -> E_P
     B_P_READY0, B_P_READY1,          // E_P done -> MMA2
     B_VH_FREE, B_VH_READY,           // decayed values: MMA4 done / E_V done
+    B_VHA_READY,                     // phase A: E_V done by the VO, P and S groups together
     B_DS_FULL, B_DS_EMPTY,           // DS: MMA4 done / E_S read it
     B_S_FREE, B_S_READY,             // state copy: MMA3 done / E_S wrote it
     B_O_FULL, B_O_EMPTY,             // OI: MMA2 done / E_O read it
@@ -680,7 +681,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
     constexpr uint64_t TILE16 = TILE_BYTES >> 4, BOX16 = BOX_BYTES >> 4;
     // nq, nkv: Q / K-V loads consumed; g: phase-C blocks; n_ds: DS productions;
     // n_vh: decayed-value tiles; n_s: state copies.
-    uint32_t nq = 0, nkv = 0, g = 0, n_ds = 0, n_vh = 0, n_s = 0;
+    uint32_t nq = 0, nkv = 0, g = 0, n_ds = 0, n_vh = 0, n_s = 0, n_vha = 0;
     auto commit = [&](int bar) {
         if (elect_one()) mma_commit(&bars[bar]);
         __syncwarp();
@@ -729,10 +730,10 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int sk = nkv & 1;
                 ok = wait_warp(&bars[B_KF0 + sk], (nkv >> 1) & 1, sm.abort, p.hdr) &&
-                     wait_warp(&bars[B_VH_READY], n_vh & 1, sm.abort, p.hdr) &&
+                     wait_warp(&bars[B_VHA_READY], n_vha & 1, sm.abort, p.hdr) &&
                      (kb > 0 || wait_warp(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr));
                 if (!ok) break;
-                ++n_vh;
+                ++n_vha;
                 tc_fence_after();
                 // In phase A, E_V (done: VH_READY) is the V slot's only reader; MMA4
                 // reads K and the decayed copy. Release the slot now, so that the
@@ -839,6 +840,46 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
     __syncwarp();
 }
 
+// Phase A (local state of a segment with a successor, or the state-only
+// pass): nothing but E_V and MMA4 runs, so the VO, P and S groups share E_V.
+// Each takes some of the 16-byte chunks of its row's 64 decayed values (VO
+// chunks 0-2, P 3-5, S 6-7) and arrives on B_VHA_READY (384 arrivals). nkv and
+// n_vh count the V loads and MMA4 completions the caller has seen.
+template <int REV>
+__device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, float slope, int row,
+                           int c0, int c1, uint32_t& nkv, uint32_t& n_vh)
+{
+    uint64_t* bars = sm.bars;
+    const int nb = num_blocks(it.len);
+    for (int kb = 0; kb < nb; ++kb) {
+        const int t0 = block_t0(it.len, kb, REV);
+        const int L = min(C, it.len - t0);
+        const int m = REV ? t0 + row : it.len - 1 - (t0 + row);
+        const int s = nkv & 1;
+        if (!wait_warp(&bars[B_VF0 + s], (nkv >> 1) & 1, sm.abort, p.hdr)) return false;
+        if (!wait_warp(&bars[B_VH_FREE], (n_vh & 1) ^ 1, sm.abort, p.hdr)) return false;
+        const float f = row < L ? expf(-slope * (float)m) : 0.f;
+        const uint64_t ff = f2(f, f);
+        const uint8_t* src = sm.v(s);
+#pragma unroll 1
+        for (int c = c0; c < c1; ++c) {
+            const uint4 u = *reinterpret_cast<const uint4*>(src + swz(row, c));
+            uint4 h, l;
+            split_pair(mul2(bf2_to_f2(u.x), ff), h.x, l.x);
+            split_pair(mul2(bf2_to_f2(u.y), ff), h.y, l.y);
+            split_pair(mul2(bf2_to_f2(u.z), ff), h.z, l.z);
+            split_pair(mul2(bf2_to_f2(u.w), ff), h.w, l.w);
+            *reinterpret_cast<uint4*>(sm.vh() + swz(row, c)) = h;
+            *reinterpret_cast<uint4*>(sm.vl() + swz(row, c)) = l;
+        }
+        fence_proxy_async();
+        mbar_arrive(&bars[B_VHA_READY]);
+        ++nkv;
+        ++n_vh;
+    }
+    return true;
+}
+
 // P group: E_P for every phase-C block.
 //
 // Full blocks take a fast path: in chunks that lie entirely on the causal
@@ -855,12 +896,17 @@ __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
     const int row = (w << 5) | lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(w << 5) << 16);
     float* pw = sm.pw;
-    uint32_t g = 0, n_sync = 0;
+    uint32_t g = 0, n_sync = 0, nkv = 0, n_vh = 0;
     Item it;
     for (uint32_t k = 0;; ++k) {
         if (!next_item(p, sm, k, it, true, lane)) break;
-        if (p.state_only) continue;  // no phase C
         const float slope = p.slopes[it.head];
+        if ((it.p_ord < it.nseg - 1 || p.state_only) &&
+            !phase_a_ev<REV>(p, sm, it, slope, row, 3, 6, nkv, n_vh))
+            break;
+        if (p.state_only) continue;  // no phase C
+        nkv += num_blocks(it.len);   // phase C: E_V is the VO group's alone
+        n_vh += num_blocks(it.len);
         if (!group_sync(&bars[B_P_SYNC], n_sync, sm.abort, p.hdr)) break;
         pw[row] = expf(-slope * (float)row);
         if (row == 0) pw[C] = expf(-slope * (float)C);
@@ -992,14 +1038,8 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
-        if (has_succ || p.state_only) {
-            for (int kb = 0; kb < nb && ok; ++kb) {
-                const int t0 = block_t0(it.len, kb, REV);
-                const int L = min(C, it.len - t0);
-                ok = e_v(slope, L, REV ? t0 + row : it.len - 1 - (t0 + row));
-            }
-            if (!ok) break;
-        }
+        if ((has_succ || p.state_only) && !phase_a_ev<REV>(p, sm, it, slope, row, 0, 3, nkv, n_vh))
+            break;
         if (p.state_only) continue;
         auto e_v_c = [&](int kb) -> bool {
             const int L = min(C, it.len - block_t0(it.len, kb, REV));
@@ -1069,7 +1109,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
     uint64_t* bars = sm.bars;
     const int a = ((warp & 3) << 5) | lane;  // TMEM lane = key dim a
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) << 5) << 16);
-    uint32_t n_ds = 0, n_s = 0, n_sync = 0;
+    uint32_t n_ds = 0, n_s = 0, n_sync = 0, nkv = 0, n_vh = 0;
     uint64_t S[DV / 2];
     Item it;
     // DS row a -> S (S = dL * S + DS when accumulate).
@@ -1127,6 +1167,12 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         const bool has_succ = it.p_ord < it.nseg - 1;
         const int chain2 = 2 * it.chain + it.half;
         bool ok = true;
+        if ((has_succ || p.state_only) && !phase_a_ev<REV>(p, sm, it, slope, a, 6, 8, nkv, n_vh))
+            break;
+        if (!p.state_only) {
+            nkv += nb;  // phase C: E_V is the VO group's alone
+            n_vh += nb;
+        }
         if (p.state_only) {
             // The chain's whole local state, plus lam^len times the incoming state.
             if (!read_ds(0.f, false)) break;
@@ -1258,6 +1304,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 i == B_S_SYNC)
                 count = 128;
             if (i == B_ITEM_EMPTY0 || i == B_ITEM_EMPTY1) count = 1 + 12;  // MMA lane + 12 group warps
+            if (i == B_VHA_READY) count = 3 * 128;  // phase-A E_V: VO, P and S groups
             mbar_init(&bars[i], count);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
