@@ -118,26 +118,30 @@ class ClockSampler:
             self.gpu = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:
             self.gpu = str(device)
+        self.err = None
         try:
             import pynvml
             pynvml.nvmlInit()
             self.handle = pynvml.nvmlDeviceGetHandleByUUID(self.gpu)
             self.nvml = pynvml
-        except Exception:
+        except Exception as e:  # noqa: BLE001 - any NVML failure selects the fallback
             self.nvml = None
+            self.err = f"nvml: {type(e).__name__}: {e}"[:200]
 
     def _run(self):
         n = self.nvml
-        max_mhz = n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM)
+        max_mhz = 0.0
         while not self.stop_flag:
             try:
+                if not max_mhz:
+                    max_mhz = n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM)
                 mhz = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
                 reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
                 watts = n.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
                 self.samples.append((time.perf_counter(), float(mhz), float(max_mhz), int(reasons),
                                      watts))
-            except Exception:
-                pass
+            except Exception as e:  # noqa: BLE001
+                self.err = f"nvml sample: {type(e).__name__}: {e}"[:200]
             time.sleep(0.001)
 
     def start(self):
@@ -164,6 +168,19 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def _snapshot(self):
+        """One nvidia-smi reading, when no sample could be taken in the loop."""
+        try:
+            out = subprocess.run(
+                ["nvidia-smi", "-i", self.gpu, "--query-gpu=clocks.sm,clocks.max.sm,"
+                 "clocks_event_reasons.sw_power_cap", "--format=csv,noheader,nounits"],
+                capture_output=True, text=True, timeout=10).stdout.strip().split(",")
+            return {"sm_mhz": float(out[0]), "sm_max_mhz": float(out[1]),
+                    "reasons": ["sw_power_cap"] if "active" in out[2].lower() else [],
+                    "samples": 1, "under_load": False, "source": "nvidia-smi, one reading after"}
+        except Exception as e:  # noqa: BLE001
+            return {"error": (self.err or "") + f"; nvidia-smi: {type(e).__name__}: {e}"[:200]}
+
     def begin(self):
         self.window = [time.perf_counter(), None]
 
@@ -182,7 +199,7 @@ class ClockSampler:
                 inside = []
             use = inside or rows
             if not use:
-                return None
+                return self._snapshot()
             reasons = sorted({name for r in use for name, bit in self.REASONS if r[3] & bit})
             return {"sm_mhz": statistics.median(r[1] for r in use),
                     "sm_mhz_min": min(r[1] for r in use),
@@ -190,7 +207,7 @@ class ClockSampler:
                     "power_w_max": round(max(r[4] for r in use), 1),
                     "samples": len(use), "under_load": bool(inside), "source": "nvml, 1 ms"}
         if self.proc is None:
-            return None
+            return self._snapshot()
         time.sleep(0.1)
         self.proc.terminate()
         try:
@@ -210,7 +227,7 @@ class ClockSampler:
                     continue
         os.unlink(self.path)
         if not rows:
-            return None
+            return self._snapshot()
         names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                  "sw_power_cap"]
         reasons = sorted({names[i] for _, _, r in rows for i in range(1, 5)
