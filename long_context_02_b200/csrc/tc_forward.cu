@@ -114,6 +114,7 @@ enum {
     B_P_READY0, B_P_READY1,          // E_P done -> MMA2
     B_VH_FREE, B_VH_READY,           // decayed values: MMA4 done / E_V done
     B_VHA_READY,                     // phase A: E_V done by the VO, P and S groups together
+    B_VH_FREE1, B_VHA_READY1,        // the second decayed-value buffer (state-only pass)
     B_DS_FULL, B_DS_EMPTY,           // DS: MMA4 done / E_S read it
     B_S_FREE, B_S_READY,             // state copy: MMA3 done / E_S wrote it
     B_O_FULL, B_O_EMPTY,             // OI: MMA2 done / E_O read it
@@ -556,6 +557,10 @@ struct Smem {
     __device__ uint8_t* vl() const { return tiles + OFF_VL; }
     __device__ uint8_t* sh() const { return tiles + OFF_SH; }
     __device__ uint8_t* sl() const { return tiles + OFF_SL; }
+    // The state-only pass loads no Q: Q slot 0 holds a second decayed-value
+    // buffer (hi, lo), so that E_V of one block overlaps MMA4 of the previous.
+    __device__ uint8_t* vh1() const { return tiles + OFF_Q; }
+    __device__ uint8_t* vl1() const { return tiles + OFF_Q + BOX_BYTES; }
 };
 
 // Reads the next item from the ring (all roles see the same sequence).
@@ -681,13 +686,14 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
     constexpr uint64_t TILE16 = TILE_BYTES >> 4, BOX16 = BOX_BYTES >> 4;
     // nq, nkv: Q / K-V loads consumed; g: phase-C blocks; n_ds: DS productions;
     // n_vh: decayed-value tiles; n_s: state copies.
-    uint32_t nq = 0, nkv = 0, g = 0, n_ds = 0, n_vh = 0, n_s = 0, n_vha = 0;
+    uint32_t nq = 0, nkv = 0, g = 0, n_ds = 0, n_vh = 0, n_s = 0, n_vha = 0, n_vha1 = 0;
+    const uint64_t dvh1 = sdesc(smem_u32(sm.vh1()), 16u, 1024u);  // second buffer (state only)
     auto commit = [&](int bar) {
         if (elect_one()) mma_commit(&bars[bar]);
         __syncwarp();
     };
-    // DS = K^T Vd (hi and lo) for the K tile in slot sk.
-    auto mma4 = [&](int sk, bool accumulate) {
+    // DS = K^T Vd (hi and lo) for the K tile in slot sk, Vd in the buffer at vd.
+    auto mma4 = [&](int sk, bool accumulate, uint64_t vd) {
         const uint64_t a = dkm0 + (uint64_t)sk * TILE16;
         const uint32_t d = tmem + COL_DS;
         const uint32_t acc0 = accumulate ? 1u : 0u;
@@ -696,7 +702,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             for (int part = 0; part < 2; ++part)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(d, a + koff_mn(ks), dvh + part * BOX16 + koff_mn(ks), IDESC_KV,
+                    mma_ss(d, a + koff_mn(ks), vd + part * BOX16 + koff_mn(ks), IDESC_KV,
                            (part || ks) ? 1u : acc0);
         }
         __syncwarp();
@@ -729,20 +735,24 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             // Phase A: DS accumulates the segment's local state over its blocks.
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int sk = nkv & 1;
+                // The state-only pass alternates the two decayed-value buffers.
+                const bool second = p.state_only && (kb & 1);
+                uint32_t& reads = second ? n_vha1 : n_vha;
                 ok = wait_warp(&bars[B_KF0 + sk], (nkv >> 1) & 1, sm.abort, p.hdr) &&
-                     wait_warp(&bars[B_VHA_READY], n_vha & 1, sm.abort, p.hdr) &&
+                     wait_warp(&bars[second ? B_VHA_READY1 : B_VHA_READY], reads & 1, sm.abort,
+                               p.hdr) &&
                      (kb > 0 || wait_warp(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr));
                 if (!ok) break;
-                ++n_vha;
+                ++reads;
                 tc_fence_after();
                 // In phase A, E_V (done: VH_READY) is the V slot's only reader; MMA4
                 // reads K and the decayed copy. Release the slot now, so that the
                 // next V load overlaps this MMA4.
                 if (elect_one()) mbar_arrive(&bars[B_VE0 + sk]);
                 __syncwarp();
-                mma4(sk, kb > 0);
+                mma4(sk, kb > 0, second ? dvh1 : dvh);
                 if (elect_one()) {
-                    mma_commit(&bars[B_VH_FREE]);
+                    mma_commit(&bars[second ? B_VH_FREE1 : B_VH_FREE]);
                     mma_commit(&bars[B_KE0 + sk]);
                 }
                 __syncwarp();
@@ -774,7 +784,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             if (!ok) break;
             ++n_vh;
             tc_fence_after();
-            mma4(skv, false);
+            mma4(skv, false, dvh);
             if (elect_one()) {
                 mma_commit(&bars[B_DS_FULL]);
                 mma_commit(&bars[B_VH_FREE]);
@@ -843,11 +853,13 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
 // Phase A (local state of a segment with a successor, or the state-only
 // pass): nothing but E_V and MMA4 runs, so the VO, P and S groups share E_V.
 // Each takes some of the 16-byte chunks of its row's 64 decayed values (VO
-// chunks 0-2, P 3-5, S 6-7) and arrives on B_VHA_READY (384 arrivals). nkv and
-// n_vh count the V loads and MMA4 completions the caller has seen.
+// chunks 0-2, P 3-5, S 6-7) and arrives on the buffer's phase-A barrier (384
+// arrivals). The state-only pass alternates between two buffers (block kb in
+// buffer kb & 1); otherwise buffer 0 alone. nkv counts the V loads the caller
+// has seen, n_vh and n_vh1 the MMA4 reads of buffers 0 and 1.
 template <int REV>
 __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, float slope, int row,
-                           int c0, int c1, uint32_t& nkv, uint32_t& n_vh)
+                           int c0, int c1, uint32_t& nkv, uint32_t& n_vh, uint32_t& n_vh1)
 {
     uint64_t* bars = sm.bars;
     const int nb = num_blocks(it.len);
@@ -856,8 +868,13 @@ __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, floa
         const int L = min(C, it.len - t0);
         const int m = REV ? t0 + row : it.len - 1 - (t0 + row);
         const int s = nkv & 1;
+        const bool second = p.state_only && (kb & 1);
+        uint32_t& uses = second ? n_vh1 : n_vh;
         if (!wait_warp(&bars[B_VF0 + s], (nkv >> 1) & 1, sm.abort, p.hdr)) return false;
-        if (!wait_warp(&bars[B_VH_FREE], (n_vh & 1) ^ 1, sm.abort, p.hdr)) return false;
+        if (!wait_warp(&bars[second ? B_VH_FREE1 : B_VH_FREE], (uses & 1) ^ 1, sm.abort, p.hdr))
+            return false;
+        uint8_t* vh = second ? sm.vh1() : sm.vh();
+        uint8_t* vl = second ? sm.vl1() : sm.vl();
         const float f = row < L ? expf(-slope * (float)m) : 0.f;
         const uint64_t ff = f2(f, f);
         const uint8_t* src = sm.v(s);
@@ -869,13 +886,13 @@ __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, floa
             split_pair(mul2(bf2_to_f2(u.y), ff), h.y, l.y);
             split_pair(mul2(bf2_to_f2(u.z), ff), h.z, l.z);
             split_pair(mul2(bf2_to_f2(u.w), ff), h.w, l.w);
-            *reinterpret_cast<uint4*>(sm.vh() + swz(row, c)) = h;
-            *reinterpret_cast<uint4*>(sm.vl() + swz(row, c)) = l;
+            *reinterpret_cast<uint4*>(vh + swz(row, c)) = h;
+            *reinterpret_cast<uint4*>(vl + swz(row, c)) = l;
         }
         fence_proxy_async();
-        mbar_arrive(&bars[B_VHA_READY]);
+        mbar_arrive(&bars[second ? B_VHA_READY1 : B_VHA_READY]);
         ++nkv;
-        ++n_vh;
+        ++uses;
     }
     return true;
 }
@@ -896,13 +913,13 @@ __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
     const int row = (w << 5) | lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(w << 5) << 16);
     float* pw = sm.pw;
-    uint32_t g = 0, n_sync = 0, nkv = 0, n_vh = 0;
+    uint32_t g = 0, n_sync = 0, nkv = 0, n_vh = 0, n_vh1 = 0;
     Item it;
     for (uint32_t k = 0;; ++k) {
         if (!next_item(p, sm, k, it, true, lane)) break;
         const float slope = p.slopes[it.head];
         if ((it.p_ord < it.nseg - 1 || p.state_only) &&
-            !phase_a_ev<REV>(p, sm, it, slope, row, 3, 6, nkv, n_vh))
+            !phase_a_ev<REV>(p, sm, it, slope, row, 3, 6, nkv, n_vh, n_vh1))
             break;
         if (p.state_only) continue;  // no phase C
         nkv += num_blocks(it.len);   // phase C: E_V is the VO group's alone
@@ -1002,7 +1019,7 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
     const int w = warp & 3;
     const int row = (w << 5) | lane;  // E_V: token row of the V tile; E_O: output row
     const uint32_t lane_addr = tmem + ((uint32_t)(w << 5) << 16);
-    uint32_t nkv = 0, n_vh = 0, g = 0;
+    uint32_t nkv = 0, n_vh = 0, n_vh1 = 0, g = 0;
     Item it;
     // E_V for the block at segment offset t0 with L valid tokens; the value
     // of token j is scaled by lam^m(j) (0 for j >= L).
@@ -1038,7 +1055,8 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
-        if ((has_succ || p.state_only) && !phase_a_ev<REV>(p, sm, it, slope, row, 0, 3, nkv, n_vh))
+        if ((has_succ || p.state_only) &&
+            !phase_a_ev<REV>(p, sm, it, slope, row, 0, 3, nkv, n_vh, n_vh1))
             break;
         if (p.state_only) continue;
         auto e_v_c = [&](int kb) -> bool {
@@ -1109,7 +1127,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
     uint64_t* bars = sm.bars;
     const int a = ((warp & 3) << 5) | lane;  // TMEM lane = key dim a
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) << 5) << 16);
-    uint32_t n_ds = 0, n_s = 0, n_sync = 0, nkv = 0, n_vh = 0;
+    uint32_t n_ds = 0, n_s = 0, n_sync = 0, nkv = 0, n_vh = 0, n_vh1 = 0;
     uint64_t S[DV / 2];
     Item it;
     // DS row a -> S (S = dL * S + DS when accumulate).
@@ -1167,7 +1185,8 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         const bool has_succ = it.p_ord < it.nseg - 1;
         const int chain2 = 2 * it.chain + it.half;
         bool ok = true;
-        if ((has_succ || p.state_only) && !phase_a_ev<REV>(p, sm, it, slope, a, 6, 8, nkv, n_vh))
+        if ((has_succ || p.state_only) &&
+            !phase_a_ev<REV>(p, sm, it, slope, a, 6, 8, nkv, n_vh, n_vh1))
             break;
         if (!p.state_only) {
             nkv += nb;  // phase C: E_V is the VO group's alone
@@ -1304,7 +1323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 i == B_S_SYNC)
                 count = 128;
             if (i == B_ITEM_EMPTY0 || i == B_ITEM_EMPTY1) count = 1 + 12;  // MMA lane + 12 group warps
-            if (i == B_VHA_READY) count = 3 * 128;  // phase-A E_V: VO, P and S groups
+            if (i == B_VHA_READY || i == B_VHA_READY1) count = 3 * 128;  // phase-A E_V: VO, P, S
             mbar_init(&bars[i], count);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
