@@ -692,8 +692,10 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         if (elect_one()) mma_commit(&bars[bar]);
         __syncwarp();
     };
-    // DS = K^T Vd (hi and lo) for the K tile in slot sk, Vd in the buffer at vd.
-    auto mma4 = [&](int sk, bool accumulate, uint64_t vd) {
+    // DS = K^T Vd (hi and lo) for the K tile in slot sk; mma4b reads the second
+    // decayed-value buffer (state-only pass). Two copies keep the descriptor of
+    // the common case a constant in the issue loop.
+    auto mma4 = [&](int sk, bool accumulate) {
         const uint64_t a = dkm0 + (uint64_t)sk * TILE16;
         const uint32_t d = tmem + COL_DS;
         const uint32_t acc0 = accumulate ? 1u : 0u;
@@ -702,7 +704,21 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             for (int part = 0; part < 2; ++part)
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(d, a + koff_mn(ks), vd + part * BOX16 + koff_mn(ks), IDESC_KV,
+                    mma_ss(d, a + koff_mn(ks), dvh + part * BOX16 + koff_mn(ks), IDESC_KV,
+                           (part || ks) ? 1u : acc0);
+        }
+        __syncwarp();
+    };
+    auto mma4b = [&](int sk, bool accumulate) {
+        const uint64_t a = dkm0 + (uint64_t)sk * TILE16;
+        const uint32_t d = tmem + COL_DS;
+        const uint32_t acc0 = accumulate ? 1u : 0u;
+        if (elect_one()) {
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_ss(d, a + koff_mn(ks), dvh1 + part * BOX16 + koff_mn(ks), IDESC_KV,
                            (part || ks) ? 1u : acc0);
         }
         __syncwarp();
@@ -750,7 +766,10 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
                 // next V load overlaps this MMA4.
                 if (elect_one()) mbar_arrive(&bars[B_VE0 + sk]);
                 __syncwarp();
-                mma4(sk, kb > 0, second ? dvh1 : dvh);
+                if (second)
+                    mma4b(sk, kb > 0);
+                else
+                    mma4(sk, kb > 0);
                 if (elect_one()) {
                     mma_commit(&bars[second ? B_VH_FREE1 : B_VH_FREE]);
                     mma_commit(&bars[B_KE0 + sk]);
@@ -784,7 +803,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             if (!ok) break;
             ++n_vh;
             tc_fence_after();
-            mma4(skv, false, dvh);
+            mma4(skv, false);
             if (elect_one()) {
                 mma_commit(&bars[B_DS_FULL]);
                 mma_commit(&bars[B_VH_FREE]);
