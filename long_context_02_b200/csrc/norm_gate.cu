@@ -14,24 +14,26 @@
 // H heads, which the prefill produces in H different CTAs at different times,
 // so it runs as its own streaming pass rather than in the prefill's epilogue.
 //
-// One CTA of 512 threads takes T consecutive tokens. Thread t owns the
-// 8-element chunks t, t + 512, ... (MAXC of them) of each token's H*d
+// One CTA of NT threads takes T consecutive tokens. Thread t owns the
+// 8-element chunks t, t + NT, ... (MAXC of them) of each token's H*d
 // features; a chunk never crosses a head row, since d is a multiple of 8.
-// T * MAXC = 4 keeps the registers per thread fixed, and T is as large as
-// the feature count allows (H*d <= 4096: T = 4; <= 8192: T = 2; <= 16384:
-// T = 1), so each CTA has T tokens' O and G in flight at once. All loads are
-// issued, with streaming hints, before the reduction; the block reduces the
-// T sums of squares in a fixed order under one barrier, then every thread
-// scales, gates and stores its chunks. Bytes per token: H*d*(|O| + 2|Y|)
-// plus w, which stays in L2. The gate uses the fast exponential and division
-// intrinsics, so the arithmetic stays well under the memory time.
+// T * MAXC = 4 keeps the registers per thread fixed. CTAs are kept small
+// (NT = 256 up to H*d = 8192, with T = 4, 2, 1 as H*d grows; NT = 512 and
+// T = 1 up to 16384) so that five of them share an SM: each CTA waits at
+// its one barrier at a different time, and the SM always has loads in
+// flight. All loads are issued, with streaming hints, before the reduction;
+// the block reduces the T sums of squares in a fixed order under one
+// barrier, then every thread scales, gates and stores its chunks. Bytes per
+// token: H*d*(|O| + 2|Y|) plus w, which stays in L2. The gate uses the fast
+// exponential and division intrinsics, so the arithmetic stays well under
+// the memory time.
 #include "kernels.h"
 
 namespace la {
 namespace {
 
-constexpr int NG_THREADS = 512;
-constexpr int NG_SLOTS = 4;  // T * MAXC: H*d <= 512 * 8 * 4 / T
+constexpr int NG_THREADS_MAX = 512;
+constexpr int NG_SLOTS = 4;  // T * MAXC: H*d <= NT * 8 * 4 / T
 
 // Eight consecutive elements held in their storage type.
 template <typename T> struct Chunk8;
@@ -80,8 +82,8 @@ template <> struct Chunk8<float> {
 // intrinsics (a few ulp; a large negative x gives e^-x = inf and a gate of 0).
 __device__ __forceinline__ float sigmoid(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
-template <typename To, typename Tg, int T>
-__global__ void __launch_bounds__(NG_THREADS) norm_gate_kernel(const To* __restrict__ o,
+template <typename To, typename Tg, int NT, int T>
+__global__ void __launch_bounds__(NT) norm_gate_kernel(const To* __restrict__ o,
                                                                const Tg* __restrict__ g,
                                                                const float* __restrict__ w,
                                                                float eps, Tg* __restrict__ y,
@@ -89,7 +91,7 @@ __global__ void __launch_bounds__(NG_THREADS) norm_gate_kernel(const To* __restr
                                                                long long tokens)
 {
     constexpr int MAXC = NG_SLOTS / T;
-    __shared__ float red[T][NG_THREADS / 32];
+    __shared__ float red[T][NT / 32];
     const long long t0 = (long long)blockIdx.x * T;
     const int F = H * d, nchunks = F / 8, cpr = d / 8;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(NG_THREADS) norm_gate_kernel(const To* __restr
         const long long b = t / N, n = t % N;
 #pragma unroll
         for (int m = 0; m < MAXC; ++m) {
-            const int c = tid + NG_THREADS * m;
+            const int c = tid + NT * m;
             if (c < nchunks) {
                 const int h = c / cpr, col = (c - h * cpr) * 8;
                 xo[j][m].load(o + ((b * H + h) * N + n) * d + col);
@@ -117,7 +119,7 @@ __global__ void __launch_bounds__(NG_THREADS) norm_gate_kernel(const To* __restr
         if (t0 + j < tokens) {
 #pragma unroll
             for (int m = 0; m < MAXC; ++m) {
-                if (tid + NG_THREADS * m < nchunks) {
+                if (tid + NT * m < nchunks) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) ss = fmaf(xo[j][m].get(e), xo[j][m].get(e), ss);
                 }
@@ -134,11 +136,11 @@ __global__ void __launch_bounds__(NG_THREADS) norm_gate_kernel(const To* __restr
         if (t >= tokens) continue;
         float tot = 0.f;
 #pragma unroll
-        for (int i = 0; i < NG_THREADS / 32; ++i) tot += red[j][i];
+        for (int i = 0; i < NT / 32; ++i) tot += red[j][i];
         const float r = rsqrtf(tot / (float)F + eps);
 #pragma unroll
         for (int m = 0; m < MAXC; ++m) {
-            const int c = tid + NG_THREADS * m;
+            const int c = tid + NT * m;
             if (c < nchunks) {
                 const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + 8 * c));
                 const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + 8 * c) + 1);
@@ -153,12 +155,12 @@ __global__ void __launch_bounds__(NG_THREADS) norm_gate_kernel(const To* __restr
     }
 }
 
-template <typename To, typename Tg, int T>
+template <typename To, typename Tg, int NT, int T>
 cudaError_t launch_t(const void* o, const void* g, const float* w, float eps, void* y,
                      long long tokens, int H, long long N, int d, cudaStream_t stream)
 {
     const long long grid = (tokens + T - 1) / T;
-    norm_gate_kernel<To, Tg, T><<<(unsigned)grid, NG_THREADS, 0, stream>>>(
+    norm_gate_kernel<To, Tg, NT, T><<<(unsigned)grid, NT, 0, stream>>>(
         (const To*)o, (const Tg*)g, w, eps, (Tg*)y, H, N, d, tokens);
     count_launch();
     return cudaGetLastError();
@@ -171,16 +173,17 @@ cudaError_t launch(const void* o, const void* g, const float* w, float eps, void
     const long long tokens = (long long)B * N;
     if (tokens == 0) return cudaSuccess;
     const long long F = (long long)H * d;
-    if (F <= NG_THREADS * 8) return launch_t<To, Tg, 4>(o, g, w, eps, y, tokens, H, N, d, stream);
-    if (F <= NG_THREADS * 16) return launch_t<To, Tg, 2>(o, g, w, eps, y, tokens, H, N, d, stream);
-    return launch_t<To, Tg, 1>(o, g, w, eps, y, tokens, H, N, d, stream);
+    if (F <= 256 * 8) return launch_t<To, Tg, 256, 4>(o, g, w, eps, y, tokens, H, N, d, stream);
+    if (F <= 256 * 16) return launch_t<To, Tg, 256, 2>(o, g, w, eps, y, tokens, H, N, d, stream);
+    if (F <= 256 * 32) return launch_t<To, Tg, 256, 1>(o, g, w, eps, y, tokens, H, N, d, stream);
+    return launch_t<To, Tg, 512, 1>(o, g, w, eps, y, tokens, H, N, d, stream);
 }
 
 }  // namespace
 
 bool norm_gate_supported(int H, int d)
 {
-    return (long long)H * d <= (long long)NG_THREADS * NG_SLOTS * 8;
+    return (long long)H * d <= (long long)NG_THREADS_MAX * NG_SLOTS * 8;
 }
 
 cudaError_t launch_norm_gate(const void* o, const void* g, const float* w, float eps, void* y,

@@ -35,7 +35,7 @@ def _check(y, ref, y_dtype, what):
 
 @pytest.mark.parametrize("y_dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("o_dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("H,d", [(3, 64), (4, 128), (64, 128), (128, 128)])
+@pytest.mark.parametrize("H,d", [(3, 64), (4, 128), (24, 128), (64, 128), (96, 128), (128, 128)])
 def test_norm_gate(H, d, o_dtype, y_dtype):
     B, N = 2, 37
     o, gate, w = _operands(B, H, N, d, o_dtype, y_dtype, seed=H * d)
