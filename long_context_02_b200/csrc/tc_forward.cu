@@ -99,6 +99,7 @@ constexpr uint32_t OFF_SL = OFF_SH + BOX_BYTES;        // state copy, lo
 constexpr uint32_t SMEM_TILES = OFF_SL + BOX_BYTES;    // 224 KB
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_SP = 0, COL_OI = 256, COL_DS = 320, COL_OE = 384;  // OE: 128 columns
+constexpr int PREFETCH_AHEAD = 3;  // phase A: blocks between an L2 prefetch and its load
 constexpr unsigned long long WAIT_LIMIT_NS = 4000000000ull;
 constexpr unsigned long long FLAG_LIMIT_NS = 2000000000ull;
 constexpr unsigned long long DRAIN_LIMIT_NS = 200000000ull;
@@ -319,6 +320,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)),
         "l"(policy)
+        : "memory");
+}
+
+// Brings a tile into L2 ahead of its load (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z,
+                                                uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], %4;" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(z), "l"(policy)
         : "memory");
 }
 
@@ -615,6 +627,17 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int y = it.y0 + block_t0(it.len, kb, p.reverse);
                 const int s = nk & 1;
+                // Phase A's blocks are short (E_V and MMA4 only), and two slots
+                // per tile then cover less than the DRAM latency: bring the
+                // tiles of a later block into L2 first. (In phase C the same
+                // prefetch costs more than it saves.)
+                if (pass == 0 && kb + PREFETCH_AHEAD < nb && elect_one()) {
+                    const int yp = it.y0 + block_t0(it.len, kb + PREFETCH_AHEAD, p.reverse);
+                    tma_prefetch_3d(tk, 0, yp, it.z, kpol);
+                    tma_prefetch_3d(tk, 64, yp, it.z, kpol);
+                    tma_prefetch_3d(tv, DV * it.half, yp, it.z, normal);
+                }
+                __syncwarp();
                 ok = wait_warp(&bars[B_KE0 + s], ((nk >> 1) & 1) ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
                 if (elect_one()) {
