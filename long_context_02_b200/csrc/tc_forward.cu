@@ -122,6 +122,7 @@ enum {
     B_OE_FREE,                       // OE: E_O read it (MMA3 may write it)
     B_ITEM_FULL0, B_ITEM_FULL1, B_ITEM_EMPTY0, B_ITEM_EMPTY1,
     B_FIN, B_P_SYNC, B_S_SYNC,
+    B_KF2, B_KE2, B_VF2, B_VE2,      // third K and V stage (state-only pass)
     NUM_BARS
 };
 
@@ -138,6 +139,7 @@ constexpr uint32_t IDESC_QK = idesc(128, 0, 0);  // Q K^T: both K-major
 constexpr uint32_t IDESC_PV = idesc(64, 0, 1);   // P (TMEM) V: V MN-major
 constexpr uint32_t IDESC_QS = idesc(128, 0, 1);  // Q [S_hi | S_lo]: rows = key dim, MN-major
 constexpr uint32_t IDESC_KV = idesc(64, 1, 1);   // K^T Vd: both MN-major
+constexpr uint32_t IDESC_KV2 = idesc(128, 1, 1);  // K^T [Vd_hi | Vd_lo] (state-only pass)
 
 struct Params {
     int H;
@@ -563,8 +565,13 @@ struct Smem {
     volatile int* abort;
     float* pw;       // [C+1] lam^m of the P group's current item
     __device__ uint8_t* q(int s) const { return tiles + OFF_Q + s * TILE_BYTES; }
-    __device__ uint8_t* k(int s) const { return tiles + OFF_K + s * TILE_BYTES; }
-    __device__ uint8_t* v(int s) const { return tiles + OFF_V + s * BOX_BYTES; }
+    // Stage 2 (state-only pass only) uses Q slot 1 and the state-copy buffer,
+    // which that pass leaves idle.
+    __device__ uint8_t* k(int s) const
+    {
+        return s < 2 ? tiles + OFF_K + s * TILE_BYTES : tiles + OFF_Q + TILE_BYTES;
+    }
+    __device__ uint8_t* v(int s) const { return s < 2 ? tiles + OFF_V + s * BOX_BYTES : tiles + OFF_SH; }
     __device__ uint8_t* vh() const { return tiles + OFF_VH; }
     __device__ uint8_t* vl() const { return tiles + OFF_VL; }
     __device__ uint8_t* sh() const { return tiles + OFF_SH; }
@@ -589,6 +596,14 @@ __device__ __forceinline__ bool next_item(const Params& p, const Smem& sm, uint3
     return it.valid != 0;
 }
 
+// K and V stages: two, or three in the state-only pass. Use u of a tile
+// goes to stage u % n with phase (u / n) & 1.
+__device__ __forceinline__ uint32_t num_stages(const Params& p) { return p.state_only ? 3u : 2u; }
+__device__ __forceinline__ int kf_bar(uint32_t s) { return s < 2 ? B_KF0 + (int)s : B_KF2; }
+__device__ __forceinline__ int ke_bar(uint32_t s) { return s < 2 ? B_KE0 + (int)s : B_KE2; }
+__device__ __forceinline__ int vf_bar(uint32_t s) { return s < 2 ? B_VF0 + (int)s : B_VF2; }
+__device__ __forceinline__ int ve_bar(uint32_t s) { return s < 2 ? B_VE0 + (int)s : B_VE2; }
+
 // Producer warp: TMA loads (one elected lane issues; the warp waits together).
 __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUtensorMap* tk,
                               const CUtensorMap* tv, const Smem& sm, int lane)
@@ -602,6 +617,7 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
                    drop = l2_policy_evict_first();
     // nk, nv, nq: K, V and Q loads issued (K and V always come in pairs).
     uint32_t nq = 0, nk = 0, nv = 0;
+    const uint32_t NS = num_stages(p);
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
         const int slot = k & 1;
@@ -626,7 +642,7 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
             const uint64_t kpol = again ? keep : normal, vpol = again ? keep : drop;
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int y = it.y0 + block_t0(it.len, kb, p.reverse);
-                const int s = nk & 1;
+                const uint32_t s = nk % NS, ph = (nk / NS) & 1;
                 // Phase A's blocks are short (E_V and MMA4 only), and two slots
                 // per tile then cover less than the DRAM latency: bring the
                 // tiles of a later block into L2 first. (In phase C the same
@@ -638,12 +654,12 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
                     tma_prefetch_3d(tv, DV * it.half, yp, it.z, normal);
                 }
                 __syncwarp();
-                ok = wait_warp(&bars[B_KE0 + s], ((nk >> 1) & 1) ^ 1, sm.abort, p.hdr);
+                ok = wait_warp(&bars[ke_bar(s)], ph ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
                 if (elect_one()) {
-                    mbar_expect_tx(&bars[B_KF0 + s], TILE_BYTES);
-                    tma_load_3d(sm.k(s), tk, &bars[B_KF0 + s], 0, y, it.z, kpol);
-                    tma_load_3d(sm.k(s) + BOX_BYTES, tk, &bars[B_KF0 + s], 64, y, it.z, kpol);
+                    mbar_expect_tx(&bars[kf_bar(s)], TILE_BYTES);
+                    tma_load_3d(sm.k(s), tk, &bars[kf_bar(s)], 0, y, it.z, kpol);
+                    tma_load_3d(sm.k(s) + BOX_BYTES, tk, &bars[kf_bar(s)], 64, y, it.z, kpol);
                 }
                 __syncwarp();
                 ++nk;
@@ -659,11 +675,11 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
                     __syncwarp();
                     ++nq;
                 }
-                ok = wait_warp(&bars[B_VE0 + s], ((nv >> 1) & 1) ^ 1, sm.abort, p.hdr);
+                ok = wait_warp(&bars[ve_bar(s)], ((nv / NS) & 1) ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
                 if (elect_one()) {
-                    mbar_expect_tx(&bars[B_VF0 + s], BOX_BYTES);
-                    tma_load_3d(sm.v(s), tv, &bars[B_VF0 + s], DV * it.half, y, it.z, vpol);
+                    mbar_expect_tx(&bars[vf_bar(s)], BOX_BYTES);
+                    tma_load_3d(sm.v(s), tv, &bars[vf_bar(s)], DV * it.half, y, it.z, vpol);
                 }
                 __syncwarp();
                 ++nv;
@@ -674,10 +690,10 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
         // Wind down: let this CTA's copies in flight land before it exits
         // (the last use of each slot; earlier uses completed before it).
         volatile int never = 0;
-        for (uint32_t u = (nk > 2 ? nk - 2 : 0); u < nk; ++u)
-            mbar_wait(&bars[B_KF0 + (u & 1)], (u >> 1) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
-        for (uint32_t u = (nv > 2 ? nv - 2 : 0); u < nv; ++u)
-            mbar_wait(&bars[B_VF0 + (u & 1)], (u >> 1) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
+        for (uint32_t u = (nk > NS ? nk - NS : 0); u < nk; ++u)
+            mbar_wait(&bars[kf_bar(u % NS)], (u / NS) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
+        for (uint32_t u = (nv > NS ? nv - NS : 0); u < nv; ++u)
+            mbar_wait(&bars[vf_bar(u % NS)], (u / NS) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
         for (uint32_t u = (nq > 2 ? nq - 2 : 0); u < nq; ++u)
             mbar_wait(&bars[B_QF0 + (u & 1)], (u >> 1) & 1, &never, p.hdr, DRAIN_LIMIT_NS);
     }
@@ -715,9 +731,9 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         if (elect_one()) mma_commit(&bars[bar]);
         __syncwarp();
     };
-    // DS = K^T Vd (hi and lo) for the K tile in slot sk; mma4b reads the second
-    // decayed-value buffer (state-only pass). Two copies keep the descriptor of
-    // the common case a constant in the issue loop.
+    // DS = K^T Vd (hi and lo) for the K tile in slot sk. The state-only pass
+    // uses mma4s (three K stages, two decayed-value buffers); keeping this
+    // copy separate keeps its descriptors constants in the issue loop.
     auto mma4 = [&](int sk, bool accumulate) {
         const uint64_t a = dkm0 + (uint64_t)sk * TILE16;
         const uint32_t d = tmem + COL_DS;
@@ -732,17 +748,22 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         }
         __syncwarp();
     };
-    auto mma4b = [&](int sk, bool accumulate) {
-        const uint64_t a = dkm0 + (uint64_t)sk * TILE16;
-        const uint32_t d = tmem + COL_DS;
+    // The state-only pass: K stage sk of three, decayed-value buffer vb.
+    const uint64_t dkm2 = sdesc(smem_u32(sm.k(2)), BOX_BYTES, 1024u);
+    // One N = 128 MMA per k-step over [Vd_hi | Vd_lo] (adjacent boxes), so K^T
+    // is read once; the two 64-column halves accumulate apart in the score
+    // columns, which the state-only pass leaves free, and E_S adds them.
+    const uint64_t dvp = sdesc(smem_u32(sm.vh()), BOX_BYTES, 1024u);
+    const uint64_t dvp1 = sdesc(smem_u32(sm.vh1()), BOX_BYTES, 1024u);
+    auto mma4s = [&](uint32_t sk, int vb, bool accumulate) {
+        const uint64_t a = sk == 2 ? dkm2 : dkm0 + (uint64_t)sk * TILE16;
+        const uint64_t b = vb ? dvp1 : dvp;
+        const uint32_t d = tmem + COL_SP;
         const uint32_t acc0 = accumulate ? 1u : 0u;
         if (elect_one()) {
 #pragma unroll
-            for (int part = 0; part < 2; ++part)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_ss(d, a + koff_mn(ks), dvh1 + part * BOX16 + koff_mn(ks), IDESC_KV,
-                           (part || ks) ? 1u : acc0);
+            for (int ks = 0; ks < 8; ++ks)
+                mma_ss(d, a + koff_mn(ks), b + koff_mn(ks), IDESC_KV2, ks ? 1u : acc0);
         }
         __syncwarp();
     };
@@ -772,12 +793,13 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         bool ok = true;
         if (has_succ || p.state_only) {
             // Phase A: DS accumulates the segment's local state over its blocks.
+            const uint32_t NS = num_stages(p);
             for (int kb = 0; kb < nb && ok; ++kb) {
-                const int sk = nkv & 1;
+                const uint32_t sk = nkv % NS;
                 // The state-only pass alternates the two decayed-value buffers.
                 const bool second = p.state_only && (kb & 1);
                 uint32_t& reads = second ? n_vha1 : n_vha;
-                ok = wait_warp(&bars[B_KF0 + sk], (nkv >> 1) & 1, sm.abort, p.hdr) &&
+                ok = wait_warp(&bars[kf_bar(sk)], (nkv / NS) & 1, sm.abort, p.hdr) &&
                      wait_warp(&bars[second ? B_VHA_READY1 : B_VHA_READY], reads & 1, sm.abort,
                                p.hdr) &&
                      (kb > 0 || wait_warp(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr));
@@ -787,15 +809,15 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
                 // In phase A, E_V (done: VH_READY) is the V slot's only reader; MMA4
                 // reads K and the decayed copy. Release the slot now, so that the
                 // next V load overlaps this MMA4.
-                if (elect_one()) mbar_arrive(&bars[B_VE0 + sk]);
+                if (elect_one()) mbar_arrive(&bars[ve_bar(sk)]);
                 __syncwarp();
-                if (second)
-                    mma4b(sk, kb > 0);
+                if (p.state_only)
+                    mma4s(sk, second ? 1 : 0, kb > 0);
                 else
-                    mma4(sk, kb > 0);
+                    mma4((int)sk, kb > 0);
                 if (elect_one()) {
                     mma_commit(&bars[second ? B_VH_FREE1 : B_VH_FREE]);
-                    mma_commit(&bars[B_KE0 + sk]);
+                    mma_commit(&bars[ke_bar(sk)]);
                 }
                 __syncwarp();
                 ++nkv;
@@ -909,10 +931,10 @@ __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, floa
         const int t0 = block_t0(it.len, kb, REV);
         const int L = min(C, it.len - t0);
         const int m = REV ? t0 + row : it.len - 1 - (t0 + row);
-        const int s = nkv & 1;
+        const uint32_t NS = num_stages(p), s = nkv % NS;
         const bool second = p.state_only && (kb & 1);
         uint32_t& uses = second ? n_vh1 : n_vh;
-        if (!wait_warp(&bars[B_VF0 + s], (nkv >> 1) & 1, sm.abort, p.hdr)) return false;
+        if (!wait_warp(&bars[vf_bar(s)], (nkv / NS) & 1, sm.abort, p.hdr)) return false;
         if (!wait_warp(&bars[second ? B_VH_FREE1 : B_VH_FREE], (uses & 1) ^ 1, sm.abort, p.hdr))
             return false;
         uint8_t* vh = second ? sm.vh1() : sm.vh();
@@ -1193,6 +1215,25 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         ++n_ds;
         return true;
     };
+    // State-only pass: S = DS_hi + DS_lo (score columns 0..63 and 64..127).
+    auto read_ds_pair = [&]() -> bool {
+        if (!wait_warp(&bars[B_DS_FULL], n_ds & 1, sm.abort, p.hdr)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t rh[16], rl[16];
+            tmem_ld16(lane_addr + COL_SP + 16 * q4, rh);
+            tmem_ld16(lane_addr + COL_SP + DV + 16 * q4, rl);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+                S[8 * q4 + x] = add2(f2u(rh[2 * x], rh[2 * x + 1]), f2u(rl[2 * x], rl[2 * x + 1]));
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[B_DS_EMPTY]);
+        ++n_ds;
+        return true;
+    };
     // Row a of this half's 64 columns of the final state.
     auto write_state = [&](const Item& itm) {
         if (!p.state_out) return;
@@ -1236,7 +1277,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         }
         if (p.state_only) {
             // The chain's whole local state, plus lam^len times the incoming state.
-            if (!read_ds(0.f, false)) break;
+            if (!read_ds_pair()) break;
             if (p.state_in) {
                 const float dl = expf(-slope * (float)it.len);
                 const uint64_t dl2 = f2(dl, dl);
