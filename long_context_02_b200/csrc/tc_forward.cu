@@ -62,6 +62,13 @@
 // decayed values (hi, lo) and the state copies (hi, lo), all in the 128-byte
 // swizzled layout TMA writes.
 //
+// The state-only pass (final states, no outputs) runs phase A alone, as its
+// own instantiation of the kernel: it keeps three K and V stages (using the
+// Q slot and state-copy buffer it leaves idle), two decayed-value buffers,
+// and one N = 128 MMA4 per k-step over [Vd_hi | Vd_lo] whose halves
+// accumulate apart in the idle score columns. Phase A prefetches its K and V
+// tiles into L2 a few blocks ahead.
+//
 // Every wait is bounded: an mbarrier wait gives up after 4 s, the inter-CTA
 // wait after 2 s; either records LA_ERR_TIMEOUT in the workspace header and
 // the CTA winds down (waiting, bounded, for its own copies and MMAs in
@@ -155,8 +162,6 @@ struct Params {
     void* o;
     float* state_out;
     const float* state_in;  // [chains][D][D] state before token 0 (null: zero), forward only
-    int state_only;         // final states only: every item runs phase A alone (one
-                            // segment per chain), no outputs
     int reverse;
     WsHeader* hdr;
     int* chain_flags;   // per (chain, half): segments published so far
@@ -565,13 +570,12 @@ struct Smem {
     volatile int* abort;
     float* pw;       // [C+1] lam^m of the P group's current item
     __device__ uint8_t* q(int s) const { return tiles + OFF_Q + s * TILE_BYTES; }
-    // Stage 2 (state-only pass only) uses Q slot 1 and the state-copy buffer,
-    // which that pass leaves idle.
-    __device__ uint8_t* k(int s) const
-    {
-        return s < 2 ? tiles + OFF_K + s * TILE_BYTES : tiles + OFF_Q + TILE_BYTES;
-    }
-    __device__ uint8_t* v(int s) const { return s < 2 ? tiles + OFF_V + s * BOX_BYTES : tiles + OFF_SH; }
+    __device__ uint8_t* k(int s) const { return tiles + OFF_K + s * TILE_BYTES; }
+    __device__ uint8_t* v(int s) const { return tiles + OFF_V + s * BOX_BYTES; }
+    // The state-only pass's three K and V stages: stage 2 uses Q slot 1 and the
+    // state-copy buffer, which that pass leaves idle.
+    __device__ uint8_t* k3(uint32_t s) const { return s < 2 ? k((int)s) : tiles + OFF_Q + TILE_BYTES; }
+    __device__ uint8_t* v3(uint32_t s) const { return s < 2 ? v((int)s) : tiles + OFF_SH; }
     __device__ uint8_t* vh() const { return tiles + OFF_VH; }
     __device__ uint8_t* vl() const { return tiles + OFF_VL; }
     __device__ uint8_t* sh() const { return tiles + OFF_SH; }
@@ -598,13 +602,14 @@ __device__ __forceinline__ bool next_item(const Params& p, const Smem& sm, uint3
 
 // K and V stages: two, or three in the state-only pass. Use u of a tile
 // goes to stage u % n with phase (u / n) & 1.
-__device__ __forceinline__ uint32_t num_stages(const Params& p) { return p.state_only ? 3u : 2u; }
+template <int SO> __device__ __forceinline__ constexpr uint32_t num_stages() { return SO ? 3u : 2u; }
 __device__ __forceinline__ int kf_bar(uint32_t s) { return s < 2 ? B_KF0 + (int)s : B_KF2; }
 __device__ __forceinline__ int ke_bar(uint32_t s) { return s < 2 ? B_KE0 + (int)s : B_KE2; }
 __device__ __forceinline__ int vf_bar(uint32_t s) { return s < 2 ? B_VF0 + (int)s : B_VF2; }
 __device__ __forceinline__ int ve_bar(uint32_t s) { return s < 2 ? B_VE0 + (int)s : B_VE2; }
 
 // Producer warp: TMA loads (one elected lane issues; the warp waits together).
+template <int SO>
 __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUtensorMap* tk,
                               const CUtensorMap* tv, const Smem& sm, int lane)
 {
@@ -617,7 +622,7 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
                    drop = l2_policy_evict_first();
     // nk, nv, nq: K, V and Q loads issued (K and V always come in pairs).
     uint32_t nq = 0, nk = 0, nv = 0;
-    const uint32_t NS = num_stages(p);
+    const uint32_t NS = num_stages<SO>();
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
         const int slot = k & 1;
@@ -635,14 +640,13 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         // Phase A (pass 0) loads K and V; phase C (pass 1) loads Q, K and V.
-        const int last_pass = p.state_only ? 1 : 2;
-        for (int pass = (has_succ || p.state_only) ? 0 : 1; pass < last_pass && ok; ++pass) {
+        const int last_pass = SO ? 1 : 2;
+        for (int pass = (has_succ || SO) ? 0 : 1; pass < last_pass && ok; ++pass) {
             // (a state-only pass reads K and V once)
-            const bool again = pass == 0 && !p.state_only;
+            const bool again = pass == 0 && !SO;
             const uint64_t kpol = again ? keep : normal, vpol = again ? keep : drop;
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const int y = it.y0 + block_t0(it.len, kb, p.reverse);
-                const uint32_t s = nk % NS, ph = (nk / NS) & 1;
                 // Phase A's blocks are short (E_V and MMA4 only), and two slots
                 // per tile then cover less than the DRAM latency: bring the
                 // tiles of a later block into L2 first. (In phase C the same
@@ -654,12 +658,31 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
                     tma_prefetch_3d(tv, DV * it.half, yp, it.z, normal);
                 }
                 __syncwarp();
-                ok = wait_warp(&bars[ke_bar(s)], ph ^ 1, sm.abort, p.hdr);
+                if (SO) {
+                    // Three K and V stages.
+                    const uint32_t s3 = nk % 3, ph = (nk / 3) & 1;
+                    ok = wait_warp(&bars[ke_bar(s3)], ph ^ 1, sm.abort, p.hdr) &&
+                         wait_warp(&bars[ve_bar(s3)], ph ^ 1, sm.abort, p.hdr);
+                    if (!ok) break;
+                    if (elect_one()) {
+                        mbar_expect_tx(&bars[kf_bar(s3)], TILE_BYTES);
+                        tma_load_3d(sm.k3(s3), tk, &bars[kf_bar(s3)], 0, y, it.z, kpol);
+                        tma_load_3d(sm.k3(s3) + BOX_BYTES, tk, &bars[kf_bar(s3)], 64, y, it.z, kpol);
+                        mbar_expect_tx(&bars[vf_bar(s3)], BOX_BYTES);
+                        tma_load_3d(sm.v3(s3), tv, &bars[vf_bar(s3)], DV * it.half, y, it.z, vpol);
+                    }
+                    __syncwarp();
+                    ++nk;
+                    ++nv;
+                    continue;
+                }
+                const int s = nk & 1;
+                ok = wait_warp(&bars[B_KE0 + s], ((nk >> 1) & 1) ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
                 if (elect_one()) {
-                    mbar_expect_tx(&bars[kf_bar(s)], TILE_BYTES);
-                    tma_load_3d(sm.k(s), tk, &bars[kf_bar(s)], 0, y, it.z, kpol);
-                    tma_load_3d(sm.k(s) + BOX_BYTES, tk, &bars[kf_bar(s)], 64, y, it.z, kpol);
+                    mbar_expect_tx(&bars[B_KF0 + s], TILE_BYTES);
+                    tma_load_3d(sm.k(s), tk, &bars[B_KF0 + s], 0, y, it.z, kpol);
+                    tma_load_3d(sm.k(s) + BOX_BYTES, tk, &bars[B_KF0 + s], 64, y, it.z, kpol);
                 }
                 __syncwarp();
                 ++nk;
@@ -675,11 +698,11 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
                     __syncwarp();
                     ++nq;
                 }
-                ok = wait_warp(&bars[ve_bar(s)], ((nv / NS) & 1) ^ 1, sm.abort, p.hdr);
+                ok = wait_warp(&bars[B_VE0 + s], ((nv >> 1) & 1) ^ 1, sm.abort, p.hdr);
                 if (!ok) break;
                 if (elect_one()) {
-                    mbar_expect_tx(&bars[vf_bar(s)], BOX_BYTES);
-                    tma_load_3d(sm.v(s), tv, &bars[vf_bar(s)], DV * it.half, y, it.z, vpol);
+                    mbar_expect_tx(&bars[B_VF0 + s], BOX_BYTES);
+                    tma_load_3d(sm.v(s), tv, &bars[B_VF0 + s], DV * it.half, y, it.z, vpol);
                 }
                 __syncwarp();
                 ++nv;
@@ -712,6 +735,7 @@ __device__ __forceinline__ uint64_t koff_mn(int ks) { return (uint64_t)(ks * 128
 // converged) issues every MMA and commit, so that each commit tracks all
 // earlier MMAs. Descriptors are built once; each MMA adds a constant k-step
 // offset, which keeps the issue loop short.
+template <int SO>
 __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lane)
 {
     uint64_t* bars = sm.bars;
@@ -726,7 +750,6 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
     // nq, nkv: Q / K-V loads consumed; g: phase-C blocks; n_ds: DS productions;
     // n_vh: decayed-value tiles; n_s: state copies.
     uint32_t nq = 0, nkv = 0, g = 0, n_ds = 0, n_vh = 0, n_s = 0, n_vha = 0, n_vha1 = 0;
-    const uint64_t dvh1 = sdesc(smem_u32(sm.vh1()), 16u, 1024u);  // second buffer (state only)
     auto commit = [&](int bar) {
         if (elect_one()) mma_commit(&bars[bar]);
         __syncwarp();
@@ -749,15 +772,13 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         __syncwarp();
     };
     // The state-only pass: K stage sk of three, decayed-value buffer vb.
-    const uint64_t dkm2 = sdesc(smem_u32(sm.k(2)), BOX_BYTES, 1024u);
     // One N = 128 MMA per k-step over [Vd_hi | Vd_lo] (adjacent boxes), so K^T
     // is read once; the two 64-column halves accumulate apart in the score
     // columns, which the state-only pass leaves free, and E_S adds them.
-    const uint64_t dvp = sdesc(smem_u32(sm.vh()), BOX_BYTES, 1024u);
-    const uint64_t dvp1 = sdesc(smem_u32(sm.vh1()), BOX_BYTES, 1024u);
+    // (Its descriptors are built here, not kept live through phase C.)
     auto mma4s = [&](uint32_t sk, int vb, bool accumulate) {
-        const uint64_t a = sk == 2 ? dkm2 : dkm0 + (uint64_t)sk * TILE16;
-        const uint64_t b = vb ? dvp1 : dvp;
+        const uint64_t a = sdesc(smem_u32(sm.k3(sk)), BOX_BYTES, 1024u);
+        const uint64_t b = sdesc(smem_u32(vb ? sm.vh1() : sm.vh()), BOX_BYTES, 1024u);
         const uint32_t d = tmem + COL_SP;
         const uint32_t acc0 = accumulate ? 1u : 0u;
         if (elect_one()) {
@@ -791,13 +812,13 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
-        if (has_succ || p.state_only) {
+        if (has_succ || SO) {
             // Phase A: DS accumulates the segment's local state over its blocks.
-            const uint32_t NS = num_stages(p);
+            const uint32_t NS = num_stages<SO>();
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const uint32_t sk = nkv % NS;
                 // The state-only pass alternates the two decayed-value buffers.
-                const bool second = p.state_only && (kb & 1);
+                const bool second = SO && (kb & 1);
                 uint32_t& reads = second ? n_vha1 : n_vha;
                 ok = wait_warp(&bars[kf_bar(sk)], (nkv / NS) & 1, sm.abort, p.hdr) &&
                      wait_warp(&bars[second ? B_VHA_READY1 : B_VHA_READY], reads & 1, sm.abort,
@@ -811,7 +832,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
                 // next V load overlaps this MMA4.
                 if (elect_one()) mbar_arrive(&bars[ve_bar(sk)]);
                 __syncwarp();
-                if (p.state_only)
+                if (SO)
                     mma4s(sk, second ? 1 : 0, kb > 0);
                 else
                     mma4((int)sk, kb > 0);
@@ -826,7 +847,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             commit(B_DS_FULL);
             ++n_ds;
         }
-        if (p.state_only) continue;
+        if (SO) continue;
         // Phase C.
         const uint32_t q0 = nq, kv0 = nkv, g0 = g;
         if (!mma1(g0, q0, kv0)) break;
@@ -921,7 +942,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
 // arrivals). The state-only pass alternates between two buffers (block kb in
 // buffer kb & 1); otherwise buffer 0 alone. nkv counts the V loads the caller
 // has seen, n_vh and n_vh1 the MMA4 reads of buffers 0 and 1.
-template <int REV>
+template <int REV, int SO>
 __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, float slope, int row,
                            int c0, int c1, uint32_t& nkv, uint32_t& n_vh, uint32_t& n_vh1)
 {
@@ -931,8 +952,8 @@ __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, floa
         const int t0 = block_t0(it.len, kb, REV);
         const int L = min(C, it.len - t0);
         const int m = REV ? t0 + row : it.len - 1 - (t0 + row);
-        const uint32_t NS = num_stages(p), s = nkv % NS;
-        const bool second = p.state_only && (kb & 1);
+        const uint32_t NS = num_stages<SO>(), s = nkv % NS;
+        const bool second = SO && (kb & 1);
         uint32_t& uses = second ? n_vh1 : n_vh;
         if (!wait_warp(&bars[vf_bar(s)], (nkv / NS) & 1, sm.abort, p.hdr)) return false;
         if (!wait_warp(&bars[second ? B_VH_FREE1 : B_VH_FREE], (uses & 1) ^ 1, sm.abort, p.hdr))
@@ -941,7 +962,7 @@ __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, floa
         uint8_t* vl = second ? sm.vl1() : sm.vl();
         const float f = row < L ? expf(-slope * (float)m) : 0.f;
         const uint64_t ff = f2(f, f);
-        const uint8_t* src = sm.v(s);
+        const uint8_t* src = sm.v3(s);
 #pragma unroll 1
         for (int c = c0; c < c1; ++c) {
             const uint4 u = *reinterpret_cast<const uint4*>(src + swz(row, c));
@@ -969,7 +990,7 @@ __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, floa
 // starting from the exact table values, and always toward larger exponents,
 // so underflow only ever reaches values that are zero in fp32 anyway. The
 // diagonal chunk and partial blocks read the exact table per element.
-template <int REV>
+template <int REV, int SO>
 __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
     uint64_t* bars = sm.bars;
@@ -982,10 +1003,10 @@ __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
     for (uint32_t k = 0;; ++k) {
         if (!next_item(p, sm, k, it, true, lane)) break;
         const float slope = p.slopes[it.head];
-        if ((it.p_ord < it.nseg - 1 || p.state_only) &&
-            !phase_a_ev<REV>(p, sm, it, slope, row, 3, 6, nkv, n_vh, n_vh1))
+        if ((it.p_ord < it.nseg - 1 || SO) &&
+            !phase_a_ev<REV, SO>(p, sm, it, slope, row, 3, 6, nkv, n_vh, n_vh1))
             break;
-        if (p.state_only) continue;  // no phase C
+        if (SO) continue;  // no phase C
         nkv += num_blocks(it.len);   // phase C: E_V is the VO group's alone
         n_vh += num_blocks(it.len);
         if (!group_sync(&bars[B_P_SYNC], n_sync, sm.abort, p.hdr)) break;
@@ -1076,7 +1097,7 @@ __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
 
 // VO group: E_V (decayed values, hi and lo, for every block) and E_O (the
 // output rows of every phase-C block).
-template <int REV, int OUT_F32>
+template <int REV, int OUT_F32, int SO>
 __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
     uint64_t* bars = sm.bars;
@@ -1119,10 +1140,10 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         const int nb = num_blocks(it.len);
         const bool has_succ = it.p_ord < it.nseg - 1;
         bool ok = true;
-        if ((has_succ || p.state_only) &&
-            !phase_a_ev<REV>(p, sm, it, slope, row, 0, 3, nkv, n_vh, n_vh1))
+        if ((has_succ || SO) &&
+            !phase_a_ev<REV, SO>(p, sm, it, slope, row, 0, 3, nkv, n_vh, n_vh1))
             break;
-        if (p.state_only) continue;
+        if (SO) continue;
         auto e_v_c = [&](int kb) -> bool {
             const int L = min(C, it.len - block_t0(it.len, kb, REV));
             return e_v(slope, L, REV ? row : L - 1 - row);
@@ -1185,7 +1206,7 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
 // S group: E_S (the fp32 state, row a of this item's 128 x 64 state per
 // thread, kept as 32 f32x2 pairs), the hi/lo state copies for MMA3, and the
 // scan between segments.
-template <int REV>
+template <int REV, int SO>
 __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
     uint64_t* bars = sm.bars;
@@ -1268,14 +1289,14 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         const bool has_succ = it.p_ord < it.nseg - 1;
         const int chain2 = 2 * it.chain + it.half;
         bool ok = true;
-        if ((has_succ || p.state_only) &&
-            !phase_a_ev<REV>(p, sm, it, slope, a, 6, 8, nkv, n_vh, n_vh1))
+        if ((has_succ || SO) &&
+            !phase_a_ev<REV, SO>(p, sm, it, slope, a, 6, 8, nkv, n_vh, n_vh1))
             break;
-        if (!p.state_only) {
+        if (!SO) {
             nkv += nb;  // phase C: E_V is the VO group's alone
             n_vh += nb;
         }
-        if (p.state_only) {
+        if (SO) {
             // The chain's whole local state, plus lam^len times the incoming state.
             if (!read_ds_pair()) break;
             if (p.state_in) {
@@ -1379,7 +1400,7 @@ static_assert(sizeof(Item) * 2 <= SM_PW - SM_RING, "ring area");
 constexpr uint32_t SMEM_BYTES = SM_SMALL + 1023 + SMEM_TILES;
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
-template <int REV, int OUT_F32>
+template <int REV, int OUT_F32, int SO>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_forward_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv, const Params p)
@@ -1427,17 +1448,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_CTRL));
-        if (warp == 0) producer_role(p, &tq, &tk, &tv, sm, lane);
-        if (warp == 1) mma_role(p, sm, tmem, lane);
+        if (warp == 0) producer_role<SO>(p, &tq, &tk, &tv, sm, lane);
+        if (warp == 1) mma_role<SO>(p, sm, tmem, lane);
     } else if (warp < 8) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_P));
-        p_role<REV>(p, sm, tmem, warp, lane);
+        p_role<REV, SO>(p, sm, tmem, warp, lane);
     } else if (warp < 12) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_VO));
-        vo_role<REV, OUT_F32>(p, sm, tmem, warp, lane);
+        vo_role<REV, OUT_F32, SO>(p, sm, tmem, warp, lane);
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_S));
-        s_role<REV>(p, sm, tmem, warp, lane);
+        s_role<REV, SO>(p, sm, tmem, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -1698,7 +1719,6 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     prm.o = o;
     prm.state_out = state_out;
     prm.state_in = reverse ? nullptr : state_in;
-    prm.state_only = state_only;
     prm.reverse = reverse;
     prm.hdr = reinterpret_cast<WsHeader*>(ws);
     prm.chain_flags = reinterpret_cast<int*>(ws + w.flags);
@@ -1739,9 +1759,13 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
         return cudaGetLastError();
     };
     const bool f32 = out_t == LA_F32;
+    // The state-only pass (forward, no output rows) is its own instantiation,
+    // so that its paths add no code to the prefill's.
+    if (state_only && !reverse) return launch(tc_forward_kernel<0, 0, 1>);
+    if (state_only) return cudaErrorInvalidValue;
     if (reverse)
-        return f32 ? launch(tc_forward_kernel<1, 1>) : launch(tc_forward_kernel<1, 0>);
-    return f32 ? launch(tc_forward_kernel<0, 1>) : launch(tc_forward_kernel<0, 0>);
+        return f32 ? launch(tc_forward_kernel<1, 1, 0>) : launch(tc_forward_kernel<1, 0, 0>);
+    return f32 ? launch(tc_forward_kernel<0, 1, 0>) : launch(tc_forward_kernel<0, 0, 0>);
 }
 
 cudaError_t launch_tc_backward(const Problems& P, const void* dO, const void* q, const void* k,
