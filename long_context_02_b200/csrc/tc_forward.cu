@@ -62,8 +62,11 @@
 // decayed values (hi, lo) and the state copies (hi, lo), all in the 128-byte
 // swizzled layout TMA writes.
 //
-// The state-only pass (final states, no outputs) runs phase A alone, as its
-// own instantiation of the kernel: it keeps three K and V stages (using the
+// The kernel has three modes (template MODE): general (0), the state-only
+// pass (1), and one segment per chain (2: no phase A, no scan, used by dense
+// problems whose chains fill the GPU). Each is its own instantiation, so no
+// mode carries another's code. The state-only pass (final states, no
+// outputs) runs phase A alone: it keeps three K and V stages (using the
 // Q slot and state-copy buffer it leaves idle), two decayed-value buffers,
 // and one N = 128 MMA4 per k-step over [Vd_hi | Vd_lo] whose halves
 // accumulate apart in the idle score columns. Phase A prefetches its K and V
@@ -609,10 +612,11 @@ __device__ __forceinline__ int vf_bar(uint32_t s) { return s < 2 ? B_VF0 + (int)
 __device__ __forceinline__ int ve_bar(uint32_t s) { return s < 2 ? B_VE0 + (int)s : B_VE2; }
 
 // Producer warp: TMA loads (one elected lane issues; the warp waits together).
-template <int SO>
+template <int MODE>
 __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUtensorMap* tk,
                               const CUtensorMap* tv, const Smem& sm, int lane)
 {
+    constexpr bool SO = MODE == 1, ONE = MODE == 2;
     uint64_t* bars = sm.bars;
     const int num_items = 2 * (p.cu_seqlens ? *reinterpret_cast<volatile int*>(&p.hdr->num_items)
                                             : p.num_items_dense);
@@ -638,7 +642,7 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
         __syncwarp();
         if (!it.valid) break;
         const int nb = num_blocks(it.len);
-        const bool has_succ = it.p_ord < it.nseg - 1;
+        const bool has_succ = !ONE && it.p_ord < it.nseg - 1;
         // Phase A (pass 0) loads K and V; phase C (pass 1) loads Q, K and V.
         const int last_pass = SO ? 1 : 2;
         for (int pass = (has_succ || SO) ? 0 : 1; pass < last_pass && ok; ++pass) {
@@ -735,9 +739,10 @@ __device__ __forceinline__ uint64_t koff_mn(int ks) { return (uint64_t)(ks * 128
 // converged) issues every MMA and commit, so that each commit tracks all
 // earlier MMAs. Descriptors are built once; each MMA adds a constant k-step
 // offset, which keeps the issue loop short.
-template <int SO>
+template <int MODE>
 __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lane)
 {
+    constexpr bool SO = MODE == 1, ONE = MODE == 2;
     uint64_t* bars = sm.bars;
     // Slot s's tile is slot 0's plus a fixed distance, so one base per tensor.
     const uint64_t dq0 = sdesc(smem_u32(sm.q(0)), 16u, 1024u);
@@ -810,7 +815,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
     for (uint32_t k = 0;; ++k) {
         if (!next_item(p, sm, k, it, true, lane)) break;
         const int nb = num_blocks(it.len);
-        const bool has_succ = it.p_ord < it.nseg - 1;
+        const bool has_succ = !ONE && it.p_ord < it.nseg - 1;
         bool ok = true;
         if (has_succ || SO) {
             // Phase A: DS accumulates the segment's local state over its blocks.
@@ -942,10 +947,11 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
 // arrivals). The state-only pass alternates between two buffers (block kb in
 // buffer kb & 1); otherwise buffer 0 alone. nkv counts the V loads the caller
 // has seen, n_vh and n_vh1 the MMA4 reads of buffers 0 and 1.
-template <int REV, int SO>
+template <int REV, int MODE>
 __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, float slope, int row,
                            int c0, int c1, uint32_t& nkv, uint32_t& n_vh, uint32_t& n_vh1)
 {
+    constexpr bool SO = MODE == 1, ONE = MODE == 2;
     uint64_t* bars = sm.bars;
     const int nb = num_blocks(it.len);
     for (int kb = 0; kb < nb; ++kb) {
@@ -990,9 +996,10 @@ __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, floa
 // starting from the exact table values, and always toward larger exponents,
 // so underflow only ever reaches values that are zero in fp32 anyway. The
 // diagonal chunk and partial blocks read the exact table per element.
-template <int REV, int SO>
+template <int REV, int MODE>
 __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
+    constexpr bool SO = MODE == 1, ONE = MODE == 2;
     uint64_t* bars = sm.bars;
     const int w = warp & 3;
     const int row = (w << 5) | lane;
@@ -1003,8 +1010,8 @@ __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
     for (uint32_t k = 0;; ++k) {
         if (!next_item(p, sm, k, it, true, lane)) break;
         const float slope = p.slopes[it.head];
-        if ((it.p_ord < it.nseg - 1 || SO) &&
-            !phase_a_ev<REV, SO>(p, sm, it, slope, row, 3, 6, nkv, n_vh, n_vh1))
+        if (((!ONE && it.p_ord < it.nseg - 1) || SO) &&
+            !phase_a_ev<REV, MODE>(p, sm, it, slope, row, 3, 6, nkv, n_vh, n_vh1))
             break;
         if (SO) continue;  // no phase C
         nkv += num_blocks(it.len);   // phase C: E_V is the VO group's alone
@@ -1097,9 +1104,10 @@ __device__ void p_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
 
 // VO group: E_V (decayed values, hi and lo, for every block) and E_O (the
 // output rows of every phase-C block).
-template <int REV, int OUT_F32, int SO>
+template <int REV, int OUT_F32, int MODE>
 __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
+    constexpr bool SO = MODE == 1, ONE = MODE == 2;
     uint64_t* bars = sm.bars;
     const int w = warp & 3;
     const int row = (w << 5) | lane;  // E_V: token row of the V tile; E_O: output row
@@ -1138,10 +1146,10 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
         if (!next_item(p, sm, k, it, true, lane)) break;
         const float slope = p.slopes[it.head];
         const int nb = num_blocks(it.len);
-        const bool has_succ = it.p_ord < it.nseg - 1;
+        const bool has_succ = !ONE && it.p_ord < it.nseg - 1;
         bool ok = true;
         if ((has_succ || SO) &&
-            !phase_a_ev<REV, SO>(p, sm, it, slope, row, 0, 3, nkv, n_vh, n_vh1))
+            !phase_a_ev<REV, MODE>(p, sm, it, slope, row, 0, 3, nkv, n_vh, n_vh1))
             break;
         if (SO) continue;
         auto e_v_c = [&](int kb) -> bool {
@@ -1206,9 +1214,10 @@ __device__ void vo_role(const Params& p, const Smem& sm, uint32_t tmem, int warp
 // S group: E_S (the fp32 state, row a of this item's 128 x 64 state per
 // thread, kept as 32 f32x2 pairs), the hi/lo state copies for MMA3, and the
 // scan between segments.
-template <int REV, int SO>
+template <int REV, int MODE>
 __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp, int lane)
 {
+    constexpr bool SO = MODE == 1, ONE = MODE == 2;
     uint64_t* bars = sm.bars;
     const int a = ((warp & 3) << 5) | lane;  // TMEM lane = key dim a
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) << 5) << 16);
@@ -1286,11 +1295,11 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         if (!next_item(p, sm, k, it, true, lane)) break;
         const float slope = p.slopes[it.head];
         const int nb = num_blocks(it.len);
-        const bool has_succ = it.p_ord < it.nseg - 1;
+        const bool has_succ = !ONE && it.p_ord < it.nseg - 1;
         const int chain2 = 2 * it.chain + it.half;
         bool ok = true;
         if ((has_succ || SO) &&
-            !phase_a_ev<REV, SO>(p, sm, it, slope, a, 6, 8, nkv, n_vh, n_vh1))
+            !phase_a_ev<REV, MODE>(p, sm, it, slope, a, 6, 8, nkv, n_vh, n_vh1))
             break;
         if (!SO) {
             nkv += nb;  // phase C: E_V is the VO group's alone
@@ -1322,7 +1331,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         // Incoming state: the predecessor's inclusive prefix; for the first
         // segment the caller's state before token 0, or zero.
         const float* src = p.incl + (((size_t)chain2 * 2 + ((it.p_ord - 1) & 1)) * D + a) * DV;
-        if (it.p_ord > 0) {
+        if (!ONE && it.p_ord > 0) {
             if (a == 0) {
                 const int* flag = p.chain_flags + chain2;
                 const unsigned long long t0 = globaltimer();
@@ -1348,7 +1357,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
             const float dl = expf(-slope * (float)it.len);
             const uint64_t dl2 = f2(dl, dl);
             float* dst = p.incl + (((size_t)chain2 * 2 + (it.p_ord & 1)) * D + a) * DV;
-            const bool has_prev = it.p_ord > 0;
+            const bool has_prev = !ONE && it.p_ord > 0;
             // The caller's state may be the state_out array itself: it is read here,
             // before this chain's first publish, and written after the last segment.
             const float* s_in = (has_prev || p.state_in == nullptr)
@@ -1400,7 +1409,7 @@ static_assert(sizeof(Item) * 2 <= SM_PW - SM_RING, "ring area");
 constexpr uint32_t SMEM_BYTES = SM_SMALL + 1023 + SMEM_TILES;
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
-template <int REV, int OUT_F32, int SO>
+template <int REV, int OUT_F32, int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_forward_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv, const Params p)
@@ -1448,17 +1457,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_CTRL));
-        if (warp == 0) producer_role<SO>(p, &tq, &tk, &tv, sm, lane);
-        if (warp == 1) mma_role<SO>(p, sm, tmem, lane);
+        if (warp == 0) producer_role<MODE>(p, &tq, &tk, &tv, sm, lane);
+        if (warp == 1) mma_role<MODE>(p, sm, tmem, lane);
     } else if (warp < 8) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_P));
-        p_role<REV, SO>(p, sm, tmem, warp, lane);
+        p_role<REV, MODE>(p, sm, tmem, warp, lane);
     } else if (warp < 12) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_VO));
-        vo_role<REV, OUT_F32, SO>(p, sm, tmem, warp, lane);
+        vo_role<REV, OUT_F32, MODE>(p, sm, tmem, warp, lane);
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_S));
-        s_role<REV, SO>(p, sm, tmem, warp, lane);
+        s_role<REV, MODE>(p, sm, tmem, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -1763,6 +1772,13 @@ cudaError_t launch_tc_forward(const Problems& P, const void* q, const void* k, c
     // so that its paths add no code to the prefill's.
     if (state_only && !reverse) return launch(tc_forward_kernel<0, 0, 1>);
     if (state_only) return cudaErrorInvalidValue;
+    // One segment per chain (dense, long enough segments): no phase A and no
+    // scan, an instantiation without their code.
+    if (!varlen && prm.nseg == 1) {
+        if (reverse)
+            return f32 ? launch(tc_forward_kernel<1, 1, 2>) : launch(tc_forward_kernel<1, 0, 2>);
+        return f32 ? launch(tc_forward_kernel<0, 1, 2>) : launch(tc_forward_kernel<0, 0, 2>);
+    }
     if (reverse)
         return f32 ? launch(tc_forward_kernel<1, 1, 0>) : launch(tc_forward_kernel<1, 0, 0>);
     return f32 ? launch(tc_forward_kernel<0, 1, 0>) : launch(tc_forward_kernel<0, 0, 0>);
