@@ -951,7 +951,7 @@ template <int REV, int MODE>
 __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, float slope, int row,
                            int c0, int c1, uint32_t& nkv, uint32_t& n_vh, uint32_t& n_vh1)
 {
-    constexpr bool SO = MODE == 1, ONE = MODE == 2;
+    constexpr bool SO = MODE == 1;
     uint64_t* bars = sm.bars;
     const int nb = num_blocks(it.len);
     for (int kb = 0; kb < nb; ++kb) {
