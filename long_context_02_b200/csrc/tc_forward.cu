@@ -69,8 +69,10 @@
 // outputs) runs phase A alone: it keeps three K and V stages (using the
 // Q slot and state-copy buffer it leaves idle), two decayed-value buffers,
 // and one N = 128 MMA4 per k-step over [Vd_hi | Vd_lo] whose halves
-// accumulate apart in the idle score columns. Phase A prefetches its K and V
-// tiles into L2 a few blocks ahead.
+// accumulate apart in the idle score columns. The phase A of a segmented
+// chain does the same with two stages (its Q slot 0 holds the second
+// decayed-value buffer until phase A's MMAs are done, then phase C's Q).
+// Phase A prefetches its K and V tiles into L2 a few blocks ahead.
 //
 // Every wait is bounded: an mbarrier wait gives up after 4 s, the inter-CTA
 // wait after 2 s; either records LA_ERR_TIMEOUT in the workspace header and
@@ -133,6 +135,7 @@ enum {
     B_ITEM_FULL0, B_ITEM_FULL1, B_ITEM_EMPTY0, B_ITEM_EMPTY1,
     B_FIN, B_P_SYNC, B_S_SYNC,
     B_KF2, B_KE2, B_VF2, B_VE2,      // third K and V stage (state-only pass)
+    B_A_DONE,                        // a segment's phase A MMAs done: Q slot 0 is free again
     NUM_BARS
 };
 
@@ -625,7 +628,7 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
     const uint64_t keep = l2_policy_evict_last(), normal = l2_policy_evict_normal(),
                    drop = l2_policy_evict_first();
     // nk, nv, nq: K, V and Q loads issued (K and V always come in pairs).
-    uint32_t nq = 0, nk = 0, nv = 0;
+    uint32_t nq = 0, nk = 0, nv = 0, n_a = 0;
     const uint32_t NS = num_stages<SO>();
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
@@ -691,6 +694,12 @@ __device__ void producer_role(const Params& p, const CUtensorMap* tq, const CUte
                 __syncwarp();
                 ++nk;
                 if (pass == 1) {
+                    // Phase A kept its second decayed-value buffer in Q slot 0.
+                    if (kb == 0 && has_succ) {
+                        ok = wait_warp(&bars[B_A_DONE], n_a & 1, sm.abort, p.hdr);
+                        ++n_a;
+                        if (!ok) break;
+                    }
                     const int sq = nq & 1;
                     ok = wait_warp(&bars[B_QE0 + sq], ((nq >> 1) & 1) ^ 1, sm.abort, p.hdr);
                     if (!ok) break;
@@ -777,9 +786,9 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         __syncwarp();
     };
     // The state-only pass: K stage sk of three, decayed-value buffer vb.
-    // One N = 128 MMA per k-step over [Vd_hi | Vd_lo] (adjacent boxes), so K^T
-    // is read once; the two 64-column halves accumulate apart in the score
-    // columns, which the state-only pass leaves free, and E_S adds them.
+    // Phase A: one N = 128 MMA per k-step over [Vd_hi | Vd_lo] (adjacent
+    // boxes), so K^T is read once; the two 64-column halves accumulate apart
+    // in the score columns, free until phase C's first MMA1, and E_S adds them.
     // (Its descriptors are built here, not kept live through phase C.)
     auto mma4s = [&](uint32_t sk, int vb, bool accumulate) {
         const uint64_t a = sdesc(smem_u32(sm.k3(sk)), BOX_BYTES, 1024u);
@@ -820,10 +829,14 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         if (has_succ || SO) {
             // Phase A: DS accumulates the segment's local state over its blocks.
             const uint32_t NS = num_stages<SO>();
+            // The second decayed-value buffer is Q slot 0, which the previous
+            // item's MMA1 and MMA3 may still read: one more phase of its free
+            // barrier, completing after every MMA issued so far.
+            if (!SO) commit(B_VH_FREE1);
             for (int kb = 0; kb < nb && ok; ++kb) {
                 const uint32_t sk = nkv % NS;
-                // The state-only pass alternates the two decayed-value buffers.
-                const bool second = SO && (kb & 1);
+                // Phase A alternates the two decayed-value buffers.
+                const bool second = (kb & 1) != 0;
                 uint32_t& reads = second ? n_vha1 : n_vha;
                 ok = wait_warp(&bars[kf_bar(sk)], (nkv / NS) & 1, sm.abort, p.hdr) &&
                      wait_warp(&bars[second ? B_VHA_READY1 : B_VHA_READY], reads & 1, sm.abort,
@@ -837,10 +850,7 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
                 // next V load overlaps this MMA4.
                 if (elect_one()) mbar_arrive(&bars[ve_bar(sk)]);
                 __syncwarp();
-                if (SO)
-                    mma4s(sk, second ? 1 : 0, kb > 0);
-                else
-                    mma4((int)sk, kb > 0);
+                mma4s(sk, second ? 1 : 0, kb > 0);
                 if (elect_one()) {
                     mma_commit(&bars[second ? B_VH_FREE1 : B_VH_FREE]);
                     mma_commit(&bars[ke_bar(sk)]);
@@ -851,10 +861,14 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
             if (!ok) break;
             commit(B_DS_FULL);
             ++n_ds;
+            if (!SO) commit(B_A_DONE);  // the producer may load Q into slot 0 again
         }
         if (SO) continue;
         // Phase C.
         const uint32_t q0 = nq, kv0 = nkv, g0 = g;
+        // Phase A left the local state in the score columns: MMA1 may
+        // overwrite them once E_S has read it.
+        if (has_succ && !wait_warp(&bars[B_DS_EMPTY], (n_ds & 1) ^ 1, sm.abort, p.hdr)) break;
         if (!mma1(g0, q0, kv0)) break;
         for (int kb = 0; kb < nb && ok; ++kb) {
             const uint32_t gg = g0 + kb;
@@ -954,12 +968,13 @@ __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, floa
     constexpr bool SO = MODE == 1;
     uint64_t* bars = sm.bars;
     const int nb = num_blocks(it.len);
+    if (!SO) ++n_vh1;  // the MMA warp's extra phase for Q slot 0 (see mma_role)
     for (int kb = 0; kb < nb; ++kb) {
         const int t0 = block_t0(it.len, kb, REV);
         const int L = min(C, it.len - t0);
         const int m = REV ? t0 + row : it.len - 1 - (t0 + row);
         const uint32_t NS = num_stages<SO>(), s = nkv % NS;
-        const bool second = SO && (kb & 1);
+        const bool second = (kb & 1) != 0;
         uint32_t& uses = second ? n_vh1 : n_vh;
         if (!wait_warp(&bars[vf_bar(s)], (nkv / NS) & 1, sm.abort, p.hdr)) return false;
         if (!wait_warp(&bars[second ? B_VH_FREE1 : B_VH_FREE], (uses & 1) ^ 1, sm.abort, p.hdr))
@@ -1245,7 +1260,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
         ++n_ds;
         return true;
     };
-    // State-only pass: S = DS_hi + DS_lo (score columns 0..63 and 64..127).
+    // Phase A's local state: S = DS_hi + DS_lo (score columns 0..63 and 64..127).
     auto read_ds_pair = [&]() -> bool {
         if (!wait_warp(&bars[B_DS_FULL], n_ds & 1, sm.abort, p.hdr)) return false;
         tc_fence_after();
@@ -1323,7 +1338,7 @@ __device__ void s_role(const Params& p, const Smem& sm, uint32_t tmem, int warp,
             continue;
         }
         if (has_succ) {
-            if (!read_ds(0.f, false)) break;  // S = S_loc
+            if (!read_ds_pair()) break;  // S = S_loc
         } else {
 #pragma unroll
             for (int x = 0; x < DV / 2; ++x) S[x] = 0ull;
