@@ -8,7 +8,8 @@ import torch
 import oracle
 from long_context_02_b200 import binding as L
 from long_context_02_b200 import inputs
-from tests.gpu_util import (TOL_BF16, TOL_F32, assert_close, assert_close_bf16_out, f64, lam)
+from tests.gpu_util import (TOL_BF16, TOL_F32, assert_close, assert_close_bf16_out, assert_close_heads,
+                             f64, lam)
 
 pytestmark = pytest.mark.gpu
 
@@ -213,3 +214,17 @@ def test_backward_fp32_path():
     assert_close(f64(dq), rq, TOL_F32, "dQ")
     assert_close(f64(dk), rk, TOL_F32, "dK")
     assert_close(f64(dv), rv, TOL_F32, "dV")
+
+
+def test_bf16_many_items_per_cta_segmented():
+    """Two-block scan segments, ~10 items per CTA: every non-last segment runs a
+    phase A whose second decayed-value buffer shares Q slot 0 with phase C."""
+    q, k, v, s = inputs.prefill_inputs(2, 64, 1500, 128, torch.bfloat16, DEV, seed=70)
+    L.la_set_tuning(0, 256)
+    try:
+        o, st = _prefill(q, k, v, s, torch.float32)
+    finally:
+        L.la_set_tuning(0, 0)
+    o_ref, st_ref = oracle.recurrence(f64(q), f64(k), f64(v), lam(s))
+    assert_close_heads(f64(o), o_ref, TOL_BF16, range(64), "O", axis=1)
+    assert_close_heads(f64(st), st_ref, TOL_BF16, range(64), "state", axis=1)

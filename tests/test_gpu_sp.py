@@ -12,7 +12,7 @@ import torch
 import oracle
 from long_context_02_b200 import binding as L
 from long_context_02_b200 import inputs, sp
-from tests.gpu_util import TOL_BF16, TOL_F32, assert_close, f64, lam
+from tests.gpu_util import TOL_BF16, TOL_F32, assert_close, assert_close_heads, f64, lam
 
 pytestmark = pytest.mark.gpu
 
@@ -105,6 +105,20 @@ def test_prefill_state_only_fp32(d):
     torch.cuda.synchronize()
     _, want = oracle.forward(f64(q), f64(k), f64(v), lam(s), state_in=f64(s_in))
     assert_close(f64(st), want, TOL_F32, "state")
+
+
+def test_prefill_state_only_many_items_per_cta():
+    """384 items of five blocks on 148 SMs: the three-stage ring and the two
+    decayed-value buffers carry on across items of odd length."""
+    B, H, N, d = 3, 64, 520, 128
+    q, k, v, s = inputs.prefill_inputs(B, H, N, d, torch.bfloat16, DEV, seed=65)
+    s_in = inputs.state_inputs(B, H, d, DEV, seed=66)
+    ws = L.workspace(L.LA_OP_PREFILL, B, H, N, d)
+    st = s_in.clone()
+    L.la_prefill_state(k, v, s, st, st, ws)
+    assert L.la_read_device_status(ws) == L.LA_OK
+    _, want = oracle.recurrence(f64(q), f64(k), f64(v), lam(s), state_in=f64(s_in), want_o=False)
+    assert_close_heads(f64(st), want, TOL_BF16, range(H), "state", axis=1)
 
 
 def test_prefill_state_only_minimax_size():
