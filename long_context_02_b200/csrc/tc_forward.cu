@@ -127,7 +127,7 @@ enum {
     B_P_READY0, B_P_READY1,          // E_P done -> MMA2
     B_VH_FREE, B_VH_READY,           // decayed values: MMA4 done / E_V done
     B_VHA_READY,                     // phase A: E_V done by the VO, P and S groups together
-    B_VH_FREE1, B_VHA_READY1,        // the second decayed-value buffer (state-only pass)
+    B_VH_FREE1, B_VHA_READY1,        // the second decayed-value buffer (phase A)
     B_DS_FULL, B_DS_EMPTY,           // DS: MMA4 done / E_S read it
     B_S_FREE, B_S_READY,             // state copy: MMA3 done / E_S wrote it
     B_O_FULL, B_O_EMPTY,             // OI: MMA2 done / E_O read it
@@ -586,8 +586,9 @@ struct Smem {
     __device__ uint8_t* vl() const { return tiles + OFF_VL; }
     __device__ uint8_t* sh() const { return tiles + OFF_SH; }
     __device__ uint8_t* sl() const { return tiles + OFF_SL; }
-    // The state-only pass loads no Q: Q slot 0 holds a second decayed-value
-    // buffer (hi, lo), so that E_V of one block overlaps MMA4 of the previous.
+    // Phase A loads no Q: Q slot 0 holds a second decayed-value buffer (hi,
+    // lo), so that E_V of one block overlaps MMA4 of the previous. (A
+    // segmented chain's phase C takes the slot back once phase A is done.)
     __device__ uint8_t* vh1() const { return tiles + OFF_Q; }
     __device__ uint8_t* vl1() const { return tiles + OFF_Q + BOX_BYTES; }
 };
@@ -768,9 +769,9 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         if (elect_one()) mma_commit(&bars[bar]);
         __syncwarp();
     };
-    // DS = K^T Vd (hi and lo) for the K tile in slot sk. The state-only pass
-    // uses mma4s (three K stages, two decayed-value buffers); keeping this
-    // copy separate keeps its descriptors constants in the issue loop.
+    // Phase C: DS = K^T Vd (hi and lo) for the K tile in slot sk. Phase A uses
+    // mma4s; keeping this copy separate keeps its descriptors constants in
+    // the issue loop.
     auto mma4 = [&](int sk, bool accumulate) {
         const uint64_t a = dkm0 + (uint64_t)sk * TILE16;
         const uint32_t d = tmem + COL_DS;
@@ -785,11 +786,12 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
         }
         __syncwarp();
     };
-    // The state-only pass: K stage sk of three, decayed-value buffer vb.
-    // Phase A: one N = 128 MMA per k-step over [Vd_hi | Vd_lo] (adjacent
-    // boxes), so K^T is read once; the two 64-column halves accumulate apart
-    // in the score columns, free until phase C's first MMA1, and E_S adds them.
-    // (Its descriptors are built here, not kept live through phase C.)
+    // Phase A: K stage sk (of three in the state-only pass, else two) and
+    // decayed-value buffer vb, one N = 128 MMA per k-step over
+    // [Vd_hi | Vd_lo] (adjacent boxes), so K^T is read once; the two 64-column
+    // halves accumulate apart in the score columns, free until phase C's
+    // first MMA1, and E_S adds them. (Its descriptors are built here, not kept
+    // live through phase C.)
     auto mma4s = [&](uint32_t sk, int vb, bool accumulate) {
         const uint64_t a = sdesc(smem_u32(sm.k3(sk)), BOX_BYTES, 1024u);
         const uint64_t b = sdesc(smem_u32(vb ? sm.vh1() : sm.vh()), BOX_BYTES, 1024u);
@@ -958,9 +960,8 @@ __device__ void mma_role(const Params& p, const Smem& sm, uint32_t tmem, int lan
 // pass): nothing but E_V and MMA4 runs, so the VO, P and S groups share E_V.
 // Each takes some of the 16-byte chunks of its row's 64 decayed values (VO
 // chunks 0-2, P 3-5, S 6-7) and arrives on the buffer's phase-A barrier (384
-// arrivals). The state-only pass alternates between two buffers (block kb in
-// buffer kb & 1); otherwise buffer 0 alone. nkv counts the V loads the caller
-// has seen, n_vh and n_vh1 the MMA4 reads of buffers 0 and 1.
+// arrivals). Block kb uses buffer kb & 1. nkv counts the V loads the caller
+// has seen, n_vh and n_vh1 the phases of buffers 0 and 1's free barriers.
 template <int REV, int MODE>
 __device__ bool phase_a_ev(const Params& p, const Smem& sm, const Item& it, float slope, int row,
                            int c0, int c1, uint32_t& nkv, uint32_t& n_vh, uint32_t& n_vh1)
